@@ -1,0 +1,127 @@
+"""Pins for the oracle's router: canonical fp32 logit order, top-k selection, weights."""
+import itertools
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+from prefill_sigmoid_top_b200 import inputs
+from tests._util import bf16_bits, bits_to_f64, f32_to_bf16_bits
+
+
+def _bits(vals):
+    return f32_to_bf16_bits(np.asarray(vals, np.float32))
+
+
+def _single_logit(xv, wv, bias=0.0):
+    x = _bits(xv)[None, :]
+    w = _bits(wv)[None, :]
+    return float(oracle.router_logits(x, w, np.array([bias], np.float32))[0, 0])
+
+
+# ------------------------------------------------------------------ canonical order
+def test_tree_order_hand_case():
+    # H=256: lane l owns h = 8l..8l+7.  Partials: p0 = 2^24, p16 = 1, p8 = 1, p24 = 1.
+    # Tree: p0+p16 = 2^24+1 -> 2^24 (tie, even); p8+p24 = 2; then 2^24 + 2 exactly.
+    # (A left-to-right sum would give 2^24; the exact sum is 2^24 + 3.)
+    H = 256
+    x = np.zeros(H)
+    w = np.zeros(H)
+    x[0], w[0] = 4096.0, 4096.0       # lane 0 -> 2^24
+    x[8 * 16], w[8 * 16] = 1.0, 1.0   # lane 16
+    x[8 * 8], w[8 * 8] = 1.0, 1.0     # lane 8
+    x[8 * 24], w[8 * 24] = 1.0, 1.0   # lane 24
+    assert _single_logit(x, w) == 2.0 ** 24 + 2.0
+
+
+def test_lane_accumulates_sequentially_across_chunks():
+    # Lane 0 owns h = 0..7 and 256..263 (H=512).  Products 2^24, 1 (h=1), 1 (h=256),
+    # 1 (h=257): sequential fma in increasing h gives 2^24 at every step; summing each
+    # chunk first would give 2^24 + 2.
+    H = 512
+    x = np.zeros(H)
+    w = np.zeros(H)
+    x[0], w[0] = 4096.0, 4096.0
+    for h in (1, 256, 257):
+        x[h], w[h] = 1.0, 1.0
+    assert _single_logit(x, w) == 2.0 ** 24
+
+
+def test_fma_within_lane_and_bias_last():
+    # Lane 0: products 1, 2^-24 (h=1), then bias 2^-24.  Sequential: 1 + 2^-24 -> 1
+    # (tie, even).  Bias added after the tree: 1 + 2^-24 -> 1.  Exact would be 1 + 2^-23.
+    H = 256
+    x = np.zeros(H)
+    w = np.zeros(H)
+    x[0], w[0] = 1.0, 1.0
+    x[1], w[1] = 2.0 ** -12, 2.0 ** -12
+    assert _single_logit(x, w, bias=2.0 ** -24) == 1.0
+    # a bias large enough to register is added exactly once, at the end
+    assert _single_logit(x, w, bias=0.5) == 1.5
+
+
+def test_logit_error_bound_random():
+    cfg = inputs.CONFIGS[0].with_(M=32, H=1024, E=16)
+    w_router, bias, gamma, x = inputs.router_inputs(cfg)
+    z32, z64 = oracle.router_logits(bf16_bits(x), bf16_bits(w_router), bias.numpy(), want_f64=True)
+    xd, wd = bits_to_f64(bf16_bits(x)), bits_to_f64(bf16_bits(w_router))
+    absdot = np.abs(xd) @ np.abs(wd).T
+    bound = 2 * cfg.H * 2.0 ** -24 * absdot + np.abs(z64) * 2.0 ** -24
+    assert (np.abs(z32.astype(np.float64) - z64) <= bound).all()
+    # and the fp64 value is the plain dot product (numpy matmul as the library check)
+    assert np.allclose(z64, xd @ wd.T + bias.numpy().astype(np.float64), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ top-k
+def _valid_topk_set(z, S, K):
+    """S is the top-k set: every selected key beats every unselected one (ties -> lower id)."""
+    if len(set(S)) != K:
+        return False
+    rest = [j for j in range(len(z)) if j not in S]
+    for i in S:
+        for j in rest:
+            if not (z[i] > z[j] or (z[i] == z[j] and i < j)):
+                return False
+    return True
+
+
+def test_topk_exhaustive_tiny():
+    cfg = inputs.CONFIGS[0]
+    w_router, bias, gamma, x = inputs.router_inputs(cfg)
+    z = oracle.router_logits(bf16_bits(x), bf16_bits(w_router), bias.numpy())
+    ids, w = oracle.topk(z, cfg.K)
+    for t in range(cfg.M):
+        valid = [S for S in itertools.combinations(range(cfg.E), cfg.K) if _valid_topk_set(z[t], S, cfg.K)]
+        assert len(valid) == 1
+        assert sorted(ids[t].tolist()) == sorted(valid[0])
+        # slot order: descending key, ties to lower id
+        for a, b in zip(ids[t][:-1], ids[t][1:]):
+            assert z[t, a] > z[t, b] or (z[t, a] == z[t, b] and a < b)
+
+
+def test_topk_ties_and_signed_zero():
+    z = np.array([[0.0, -0.0, 1.0, 1.0, -0.0, 0.0, 2.0, -1.0],
+                  [-0.0, 0.0, 0.0, -0.0, -0.0, 0.0, 0.0, 0.0]], np.float32)
+    ids, w = oracle.topk(z, 5)
+    assert ids[0].tolist() == [6, 2, 3, 0, 1]
+    assert ids[1].tolist() == [0, 1, 2, 3, 4]
+    assert np.allclose(w[1], 0.2, rtol=0, atol=1e-15)
+
+
+def test_weights_sum_order_and_ratio():
+    rng = np.random.default_rng(5)
+    z = (rng.standard_normal((64, 256)) * 2).astype(np.float32)
+    K = 16
+    ids, w = oracle.topk(z, K)
+    assert np.allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert (np.diff(w, axis=1) <= 0).all()
+    sel = np.take_along_axis(z, ids, axis=1).astype(np.float64)
+    s = scipy.special.expit(sel)   # library sigmoid
+    assert np.allclose(w, s / s.sum(axis=1, keepdims=True), rtol=1e-13, atol=0)
+
+
+def test_route_all_configs_shapes_small():
+    # the canonical order needs H % 256 == 0; every workload satisfies it
+    for cfg in inputs.CONFIGS.values():
+        assert cfg.H % 256 == 0 and cfg.K <= cfg.E
