@@ -1,0 +1,284 @@
+"""Python binding of libmoe_b200.so, the B200 (sm_100a) routed-MoE layer library.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels (see include/moe_b200.h for the operations and their definitions).
+Tensors are torch CUDA tensors; the library is called on
+``torch.cuda.current_stream()``.  There is no CPU fallback: if the library
+cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "MoEError", "Shape", "library", "route", "align_block_size", "grouped_up_swiglu", "grouped_down",
+    "finalize_rmsnorm", "layer", "layer_workspace_size", "layer_workspace_layout", "align_capacity",
+    "route_workspace_size", "get_device_error", "status_string", "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_INVALID_INPUT", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_CUDA"}
+MOE_W_BF16, MOE_W_NVFP4 = 0, 1
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}" if what else status_string(status))
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("block_size", ctypes.c_int32)]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("gate", ctypes.c_void_p), ("up", ctypes.c_void_p),
+                ("down", ctypes.c_void_p), ("gate_gs", ctypes.c_void_p), ("up_gs", ctypes.c_void_p),
+                ("down_gs", ctypes.c_void_p)]
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("sorted_ids", ctypes.c_void_p), ("block_expert", ctypes.c_void_p),
+                ("expert_counts", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
+                ("num_tokens_post_padded", ctypes.c_void_p)]
+
+
+_LAYOUT_FIELDS = ["err_flag", "logits", "topk_ids", "topk_w", "sorted_ids", "block_expert", "expert_counts",
+                  "expert_offsets", "num_tokens_post_padded", "h", "y", "act_scratch", "total"]
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_size_t) for f in _LAYOUT_FIELDS]
+
+
+@dataclass(frozen=True)
+class Shape:
+    M: int
+    H: int
+    I: int
+    E: int
+    top_k: int
+    block_size: int
+
+    def c(self) -> _Shape:
+        return _Shape(self.M, self.H, self.I, self.E, self.top_k, self.block_size)
+
+
+def _declare(L):
+    vp, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    sig = {
+        "moe_status_string": (ctypes.c_char_p, [st]),
+        "moe_route": (st, [vp, vp, vp, _Shape, vp, vp, vp, sz, vp]),
+        "moe_route_workspace_size": (sz, [_Shape]),
+        "moe_align_block_size": (st, [vp, _Shape, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_align_capacity": (sz, [_Shape]),
+        "moe_grouped_up_swiglu": (st, [vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Plan), _Shape, vp, vp, sz,
+                                       vp, vp]),
+        "moe_up_workspace_size": (sz, [_Shape, ctypes.c_int]),
+        "moe_grouped_down": (st, [vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Plan), _Shape, vp, vp, sz, vp,
+                                  vp]),
+        "moe_down_workspace_size": (sz, [_Shape, ctypes.c_int]),
+        "moe_finalize_rmsnorm": (st, [vp, vp, vp, vp, ctypes.c_float, _Shape, vp, vp, vp]),
+        "moe_layer": (st, [vp, vp, vp, ctypes.POINTER(_Weights), vp, ctypes.c_float, _Shape, vp, vp, vp, vp, vp,
+                           sz, vp]),
+        "moe_layer_workspace_size": (sz, [_Shape, ctypes.c_int]),
+        "moe_layer_workspace_layout": (st, [_Shape, ctypes.c_int, ctypes.POINTER(_Layout)]),
+        "moe_quantize_nvfp4": (st, [vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, vp, vp, vp, vp, sz, vp]),
+        "moe_nvfp4_quantize_workspace_size": (sz, [ctypes.c_int64]),
+        "moe_prepare_nvfp4_weights": (st, [vp, vp, _Shape, ctypes.c_int, vp, sz, vp]),
+        "moe_nvfp4_blob_bytes": (sz, [_Shape, ctypes.c_int]),
+        "moe_get_device_error": (st, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+
+
+def library():
+    """The loaded libmoe_b200.so (built in-tree on first use if it is missing)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                from . import build as _build
+                _build.build()
+            L = ctypes.CDLL(_LIB_PATH)
+            _declare(L)
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return library().moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MoEError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("moe_b200 operates on CUDA tensors only")
+
+
+def _bf16(t):
+    if t.dtype != torch.bfloat16 or not t.is_contiguous():
+        raise ValueError("expected a contiguous bf16 tensor")
+    return t
+
+
+def _weights_struct(w_gate, w_up, w_down):
+    return _Weights(MOE_W_BF16, w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr(), None, None, None)
+
+
+# ------------------------------------------------------------------ sizes
+def align_capacity(shape: Shape) -> int:
+    return int(library().moe_align_capacity(shape.c()))
+
+
+def route_workspace_size(shape: Shape) -> int:
+    return int(library().moe_route_workspace_size(shape.c()))
+
+
+def layer_workspace_size(shape: Shape, wdtype: int = MOE_W_BF16) -> int:
+    return int(library().moe_layer_workspace_size(shape.c(), wdtype))
+
+
+def layer_workspace_layout(shape: Shape, wdtype: int = MOE_W_BF16) -> dict:
+    lay = _Layout()
+    _check(library().moe_layer_workspace_layout(shape.c(), wdtype, ctypes.byref(lay)), "moe_layer_workspace_layout")
+    return {f: int(getattr(lay, f)) for f in _LAYOUT_FIELDS}
+
+
+# ------------------------------------------------------------------ steps
+def route(x, w_router, bias, top_k, topk_ids=None, topk_w=None, ws=None):
+    """Sigmoid top-k routing -> (topk_ids int32 [M,K], topk_w fp32 [M,K])."""
+    _need_cuda(x, w_router, bias)
+    M, H = x.shape
+    E = w_router.shape[0]
+    shape = Shape(M, H, 128, E, top_k, 16)
+    if topk_ids is None:
+        topk_ids = torch.empty(M, top_k, dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty(M, top_k, dtype=torch.float32, device=x.device)
+    need = route_workspace_size(shape)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(library().moe_route(_ptr(_bf16(x)), _ptr(_bf16(w_router)), _ptr(bias), shape.c(), _ptr(topk_ids),
+                               _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_route")
+    return topk_ids, topk_w
+
+
+def align_block_size(topk_ids, E, block_size, err_flag=None, out=None):
+    """Expert-major plan -> dict of device tensors (sorted_ids, block_expert, expert_counts,
+    expert_offsets, num_tokens_post_padded)."""
+    _need_cuda(topk_ids)
+    M, K = topk_ids.shape
+    shape = Shape(M, 256, 128, E, K, block_size)
+    cap = align_capacity(shape)
+    if cap == 0:
+        raise MoEError(2, "moe_align_capacity")
+    dev = topk_ids.device
+    if out is None:
+        out = dict(sorted_ids=torch.empty(cap, dtype=torch.int32, device=dev),
+                   block_expert=torch.empty(cap // block_size + 1, dtype=torch.int32, device=dev),
+                   expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+                   expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                   num_tokens_post_padded=torch.empty(1, dtype=torch.int32, device=dev))
+    _check(library().moe_align_block_size(_ptr(topk_ids), shape.c(), _ptr(out["sorted_ids"]),
+                                          _ptr(out["block_expert"]), _ptr(out["expert_counts"]),
+                                          _ptr(out["expert_offsets"]), _ptr(out["num_tokens_post_padded"]),
+                                          _ptr(err_flag), _stream()), "moe_align_block_size")
+    return out
+
+
+def _plan_struct(plan):
+    return _Plan(plan["sorted_ids"].data_ptr(), plan["block_expert"].data_ptr(), plan["expert_counts"].data_ptr(),
+                 plan["expert_offsets"].data_ptr(), plan["num_tokens_post_padded"].data_ptr())
+
+
+def grouped_up_swiglu(x, w_gate, w_up, plan, shape: Shape, h=None, err_flag=None):
+    """h[cap, I] = bf16(silu(x W_gate^T) * (x W_up^T)) in plan order."""
+    _need_cuda(x, w_gate, w_up)
+    if h is None:
+        h = torch.empty(align_capacity(shape), shape.I, dtype=torch.bfloat16, device=x.device)
+    w = _weights_struct(w_gate, w_up, w_up)
+    p = _plan_struct(plan)
+    _check(library().moe_grouped_up_swiglu(_ptr(_bf16(x)), ctypes.byref(w), ctypes.byref(p), shape.c(), _ptr(h),
+                                           None, 0, _ptr(err_flag), _stream()), "moe_grouped_up_swiglu")
+    return h
+
+
+def grouped_down(h, w_down, plan, shape: Shape, y=None, err_flag=None):
+    """y[M*K, H] = bf16(h W_down^T), scattered to slot order."""
+    _need_cuda(h, w_down)
+    if y is None:
+        y = torch.empty(shape.M * shape.top_k, shape.H, dtype=torch.bfloat16, device=h.device)
+    w = _weights_struct(w_down, w_down, w_down)
+    p = _plan_struct(plan)
+    _check(library().moe_grouped_down(_ptr(_bf16(h)), ctypes.byref(w), ctypes.byref(p), shape.c(), _ptr(y), None, 0,
+                                      _ptr(err_flag), _stream()), "moe_grouped_down")
+    return y
+
+
+def finalize_rmsnorm(x, y, topk_w, gamma, eps, out=None, residual_out=None, want_residual=False):
+    """out = RMSNorm(x + sum_k w_k y_k) * gamma (and bf16(x + sum) if asked)."""
+    _need_cuda(x, y, topk_w, gamma)
+    M, H = x.shape
+    K = topk_w.shape[1]
+    shape = Shape(M, H, 128, max(K, 1), K, 16)
+    if out is None:
+        out = torch.empty_like(x)
+    if want_residual and residual_out is None:
+        residual_out = torch.empty_like(x)
+    _check(library().moe_finalize_rmsnorm(_ptr(_bf16(x)), _ptr(_bf16(y)), _ptr(topk_w), _ptr(_bf16(gamma)),
+                                          float(eps), shape.c(), _ptr(out), _ptr(residual_out), _stream()),
+           "moe_finalize_rmsnorm")
+    return (out, residual_out) if want_residual else out
+
+
+def layer(x, w_router, bias, w_gate, w_up, w_down, gamma, eps, top_k, block_size, ws=None, out=None,
+          residual_out=None, topk_ids=None, topk_w=None):
+    """The whole routed-MoE layer; returns out [M,H] bf16."""
+    _need_cuda(x, w_router, w_gate, w_up, w_down, gamma)
+    M, H = x.shape
+    E, I = w_gate.shape[0], w_gate.shape[1]
+    shape = Shape(M, H, I, E, top_k, block_size)
+    if ws is None:
+        ws = torch.empty(layer_workspace_size(shape), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    w = _weights_struct(w_gate, w_up, w_down)
+    _check(library().moe_layer(_ptr(_bf16(x)), _ptr(_bf16(w_router)), _ptr(bias), ctypes.byref(w),
+                               _ptr(_bf16(gamma)), float(eps), shape.c(), _ptr(out), _ptr(residual_out),
+                               _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_layer")
+    return out
+
+
+def get_device_error(err_flag) -> int:
+    """Synchronise the current stream and return the device-detected status (0 = none)."""
+    code = ctypes.c_int32(0)
+    _check(library().moe_get_device_error(_ptr(err_flag), _stream(), ctypes.byref(code)), "moe_get_device_error")
+    return int(code.value)

@@ -1,0 +1,369 @@
+// C-ABI entry points of libmoe_b200.so (declared and documented in
+// include/moe_b200.h): host-side validation, TMA tensor-map encoding,
+// workspace layout, and the launch sequence of the layer.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_b200.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using moe::GroupedGemmArgs;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+moe_status_t check_shape(const moe_shape_t& s) {
+  if (s.M < 1 || s.H < 256 || s.I < 128 || s.E < 1 || s.top_k < 1 || s.block_size < 1) return MOE_ERR_UNSUPPORTED;
+  if (s.H % 256 != 0 || s.H > 8192) return MOE_ERR_UNSUPPORTED;
+  if (s.I % 128 != 0 || s.I > 65536) return MOE_ERR_UNSUPPORTED;
+  if (s.E > 1024 || s.top_k > s.E || s.top_k > 32) return MOE_ERR_UNSUPPORTED;
+  if (!is_pow2(s.block_size) || s.block_size < 16 || s.block_size > 256) return MOE_ERR_UNSUPPORTED;
+  const long long mk = static_cast<long long>(s.M) * s.top_k;
+  const long long cap = mk + static_cast<long long>(s.E) * (s.block_size - 1);
+  if (cap >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous) read in boxes of
+// box_rows x 64 elements (128 bytes) with the 128-byte swizzle.
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Token-tile width of the grouped kernels: the mean routed rows per expert
+// decides between the decode shape (32) and the batch/prefill shape (128).
+// MOE_GEMM_NMAX=32|128 overrides (used by tests to cover both shapes).
+int choose_nmax(const moe_shape_t& s) {
+  if (const char* env = std::getenv("MOE_GEMM_NMAX")) {
+    const int v = std::atoi(env);
+    if (v == 32 || v == 128) return v;
+  }
+  const double per_expert = static_cast<double>(s.M) * s.top_k / s.E;
+  return per_expert <= 24.0 ? 32 : 128;
+}
+
+size_t cap_rows(const moe_shape_t& s) {
+  return static_cast<size_t>(s.M) * s.top_k + static_cast<size_t>(s.E) * (s.block_size - 1);
+}
+
+moe_status_t check_plan(const moe_plan_t* p) {
+  if (p == nullptr || p->sorted_ids == nullptr || p->expert_counts == nullptr || p->expert_offsets == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(p->sorted_ids)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status_t check_bf16_weights(const moe_weights_t* w) {
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (w->dtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
+                    moe_bf16_t* h, int32_t* err, cudaStream_t stream) {
+  CUtensorMap mg, mu, mx;
+  const uint64_t rows = static_cast<uint64_t>(s.E) * s.I;
+  if (!make_map_bf16(&mg, w->gate, rows, s.H, 128) || !make_map_bf16(&mu, w->up, rows, s.H, 128) ||
+      !make_map_bf16(&mx, x, s.M, s.H, 1))
+    return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.sorted_ids = plan->sorted_ids;
+  a.expert_counts = plan->expert_counts;
+  a.expert_offsets = plan->expert_offsets;
+  a.out = h;
+  a.err = err;
+  a.M = s.M;
+  a.E = s.E;
+  a.top_k = s.top_k;
+  a.rows_per_expert = s.I;
+  a.kdim = s.H;
+  a.out_ld = s.I;
+  return cuda_status(moe::launch_grouped_up(mg, mu, mx, a, choose_nmax(s), stream));
+}
+
+moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
+                      moe_bf16_t* y, int32_t* err, cudaStream_t stream) {
+  CUtensorMap md, mh;
+  if (!make_map_bf16(&md, w->down, static_cast<uint64_t>(s.E) * s.H, s.I, 128) ||
+      !make_map_bf16(&mh, h, cap_rows(s), s.I, 16))
+    return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.sorted_ids = plan->sorted_ids;
+  a.expert_counts = plan->expert_counts;
+  a.expert_offsets = plan->expert_offsets;
+  a.out = y;
+  a.err = err;
+  a.M = s.M;
+  a.E = s.E;
+  a.top_k = s.top_k;
+  a.rows_per_expert = s.H;
+  a.kdim = s.I;
+  a.out_ld = s.H;
+  return cuda_status(moe::launch_grouped_down(md, mh, a, choose_nmax(s), stream));
+}
+
+moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
+  (void)dt;
+  moe_layer_ws_layout_t L{};
+  const size_t mk = static_cast<size_t>(s.M) * s.top_k;
+  const size_t cap = cap_rows(s);
+  size_t off = 0;
+  L.err_flag = off;
+  off += kAlign;
+  L.logits = off;
+  off = align_up(off + static_cast<size_t>(s.M) * s.E * sizeof(float));
+  L.topk_ids = off;
+  off = align_up(off + mk * sizeof(int32_t));
+  L.topk_w = off;
+  off = align_up(off + mk * sizeof(float));
+  L.sorted_ids = off;
+  off = align_up(off + cap * sizeof(int32_t));
+  L.block_expert = off;
+  off = align_up(off + (cap / s.block_size + 1) * sizeof(int32_t));
+  L.expert_counts = off;
+  off = align_up(off + s.E * sizeof(int32_t));
+  L.expert_offsets = off;
+  off = align_up(off + (s.E + 1) * sizeof(int32_t));
+  L.num_tokens_post_padded = off;
+  off = align_up(off + sizeof(int32_t));
+  L.h = off;
+  off = align_up(off + cap * s.I * sizeof(uint16_t));
+  L.y = off;
+  off = align_up(off + mk * s.H * sizeof(uint16_t));
+  L.act_scratch = off;
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t st) {
+  switch (st) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape or dtype outside the accepted set";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_INVALID_INPUT: return "MOE_ERR_INVALID_INPUT: device found an expert id outside [0, E)";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded wait inside a kernel expired";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+  }
+  return "unknown moe_status_t";
+}
+
+size_t moe_align_capacity(moe_shape_t s) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return cap_rows(s);
+}
+
+size_t moe_route_workspace_size(moe_shape_t s) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return align_up(static_cast<size_t>(s.M) * s.E * sizeof(float));
+}
+
+size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return dtype == MOE_W_BF16 ? 0 : 0;
+}
+
+size_t moe_down_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return dtype == MOE_W_BF16 ? 0 : 0;
+}
+
+moe_status_t moe_route(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, moe_shape_t s,
+                       int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!x || !w_router || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_route_workspace_size(s)) return MOE_ERR_WORKSPACE;
+  auto cs = static_cast<cudaStream_t>(stream);
+  float* logits = static_cast<float*>(ws);
+  st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs));
+  if (st != MOE_OK) return st;
+  return cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, topk_ids, topk_w, cs));
+}
+
+moe_status_t moe_align_block_size(const int32_t* topk_ids, moe_shape_t s, int32_t* sorted_ids, int32_t* block_expert,
+                                  int32_t* expert_counts, int32_t* expert_offsets, int32_t* num_tokens_post_padded,
+                                  int32_t* err_flag, moe_stream_t stream) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!topk_ids || !sorted_ids || !block_expert || !expert_counts || !expert_offsets || !num_tokens_post_padded)
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_align(topk_ids, s.M, s.top_k, s.E, s.block_size, sorted_ids, block_expert,
+                                       expert_counts, expert_offsets, num_tokens_post_padded, err_flag,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
+                                   moe_shape_t s, moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err_flag,
+                                   moe_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if ((st = check_bf16_weights(w)) != MOE_OK) return st;
+  if ((st = check_plan(plan)) != MOE_OK) return st;
+  if (!x || !h || !w->gate || !w->up) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(h) || !aligned16(w->gate) || !aligned16(w->up)) return MOE_ERR_INVALID_ARG;
+  return run_up(x, w, plan, s, h, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_grouped_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, moe_shape_t s,
+                              moe_bf16_t* y, void* ws, size_t ws_bytes, int32_t* err_flag, moe_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if ((st = check_bf16_weights(w)) != MOE_OK) return st;
+  if ((st = check_plan(plan)) != MOE_OK) return st;
+  if (!h || !y || !w->down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(y) || !aligned16(w->down)) return MOE_ERR_INVALID_ARG;
+  return run_down(h, w, plan, s, y, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_finalize_rmsnorm(const moe_bf16_t* x, const moe_bf16_t* y, const float* topk_w,
+                                  const moe_bf16_t* gamma, float eps, moe_shape_t s, moe_bf16_t* out,
+                                  moe_bf16_t* residual_out, moe_stream_t stream) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!x || !y || !topk_w || !gamma || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(gamma) || !aligned16(out) ||
+      (residual_out && !aligned16(residual_out)))
+    return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_finalize(x, y, topk_w, gamma, eps, s.M, s.top_k, s.H, out, residual_out,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_layer_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return layer_layout(s, dtype).total;
+}
+
+moe_status_t moe_layer_workspace_layout(moe_shape_t s, moe_wdtype_t dtype, moe_layer_ws_layout_t* layout) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!layout) return MOE_ERR_INVALID_ARG;
+  *layout = layer_layout(s, dtype);
+  return MOE_OK;
+}
+
+moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, const moe_weights_t* w,
+                       const moe_bf16_t* gamma, float eps, moe_shape_t s, moe_bf16_t* out, moe_bf16_t* residual_out,
+                       int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if ((st = check_bf16_weights(w)) != MOE_OK) return st;
+  if (!x || !w_router || !gamma || !out || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(gamma) || !aligned16(out) || !aligned16(w->gate) ||
+      !aligned16(w->up) || !aligned16(w->down) || (residual_out && !aligned16(residual_out)))
+    return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  const moe_layer_ws_layout_t L = layer_layout(s, w->dtype);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  auto cs = static_cast<cudaStream_t>(stream);
+  auto* base = static_cast<uint8_t*>(ws);
+  auto* err = reinterpret_cast<int32_t*>(base + L.err_flag);
+  int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + L.topk_ids);
+  float* tw = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + L.topk_w);
+  auto* sorted = reinterpret_cast<int32_t*>(base + L.sorted_ids);
+  auto* bexp = reinterpret_cast<int32_t*>(base + L.block_expert);
+  auto* counts = reinterpret_cast<int32_t*>(base + L.expert_counts);
+  auto* offs = reinterpret_cast<int32_t*>(base + L.expert_offsets);
+  auto* ntpp = reinterpret_cast<int32_t*>(base + L.num_tokens_post_padded);
+  auto* h = reinterpret_cast<moe_bf16_t*>(base + L.h);
+  auto* y = reinterpret_cast<moe_bf16_t*>(base + L.y);
+
+  if ((st = cuda_status(cudaMemsetAsync(err, 0, sizeof(int32_t), cs))) != MOE_OK) return st;
+  float* logits = reinterpret_cast<float*>(base + L.logits);
+  if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
+    return st;
+  if ((st = cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, ids, tw, cs))) != MOE_OK) return st;
+  if ((st = cuda_status(moe::launch_align(ids, s.M, s.top_k, s.E, s.block_size, sorted, bexp, counts, offs, ntpp,
+                                          err, cs))) != MOE_OK)
+    return st;
+  moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
+  if ((st = run_up(x, w, &plan, s, h, err, cs)) != MOE_OK) return st;
+  if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
+  return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
+}
+
+moe_status_t moe_quantize_nvfp4(const moe_bf16_t* src, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* codes,
+                                uint8_t* scales, float* gs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  (void)src; (void)n_mats; (void)rows; (void)cols; (void)codes; (void)scales; (void)gs; (void)ws; (void)ws_bytes;
+  (void)stream;
+  return MOE_ERR_UNSUPPORTED;
+}
+
+size_t moe_nvfp4_quantize_workspace_size(int64_t n_mats) { return align_up(static_cast<size_t>(n_mats) * 4); }
+
+moe_status_t moe_prepare_nvfp4_weights(const uint8_t* codes, const uint8_t* scales, moe_shape_t s, int which,
+                                       void* blob, size_t blob_bytes, moe_stream_t stream) {
+  (void)codes; (void)scales; (void)s; (void)which; (void)blob; (void)blob_bytes; (void)stream;
+  return MOE_ERR_UNSUPPORTED;
+}
+
+size_t moe_nvfp4_blob_bytes(moe_shape_t s, int which) {
+  (void)s;
+  (void)which;
+  return 0;
+}
+
+moe_status_t moe_get_device_error(const int32_t* err_flag, moe_stream_t stream, int32_t* host_code) {
+  if (!err_flag || !host_code) return MOE_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, err_flag, sizeof(v), cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (v & moe::kErrTimeout)
+    *host_code = MOE_ERR_TIMEOUT;
+  else if (v & moe::kErrInvalidInput)
+    *host_code = MOE_ERR_INVALID_INPUT;
+  else
+    *host_code = MOE_OK;
+  return MOE_OK;
+}
+
+}  // extern "C"

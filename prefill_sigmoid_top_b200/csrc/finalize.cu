@@ -1,0 +1,121 @@
+// Top-k weighted sum + residual add + RMSNorm in one pass ("[flashinfer]
+// Kimi K3를 위한 초고속 통신 최적화", flashinfer PR #5701 analysis: the MoE
+// finalize fused with RMSNorm; §2 HT preset: one 128-thread consumer group per
+// token, 7 vectors of bf16x8 per thread = 896 packs = one H=7168 row; §3:
+// RMS_EPS = 1e-5 and WEIGHT_BIAS = 0, so gamma multiplies as is).
+//
+// One CTA of 128 threads per token.  Each thread owns up to 8 packs of 8
+// hidden elements (p = tid + 128*i), keeps s = x + sum_k w_k * y_k for them
+// in 64 fp32 registers, and only out (and optionally bf16(s)) is written:
+// the expert sum never goes back to HBM before the norm.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kMaxPacks = 8;  // H <= 8 * 8 * 128 = 8192
+
+__device__ __forceinline__ uint4 ld_stream_16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+  f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+  f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+  f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+__global__ void __launch_bounds__(kThreads) finalize_kernel(const uint16_t* __restrict__ x,
+                                                            const uint16_t* __restrict__ y,
+                                                            const float* __restrict__ topk_w,
+                                                            const uint16_t* __restrict__ gamma, float eps, int K,
+                                                            int H, uint16_t* __restrict__ out,
+                                                            uint16_t* __restrict__ residual_out) {
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int npk = H / 8;
+  float acc[kMaxPacks][8];
+
+#pragma unroll
+  for (int i = 0; i < kMaxPacks; ++i) {
+    const int p = tid + kThreads * i;
+    if (p < npk) {
+      unpack8(ld_stream_16(x + static_cast<size_t>(t) * H + p * 8), acc[i]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    }
+  }
+  const uint16_t* yt = y + static_cast<size_t>(t) * K * H;
+#pragma unroll 2
+  for (int k = 0; k < K; ++k) {
+    const float wk = topk_w[static_cast<size_t>(t) * K + k];
+    uint4 v[kMaxPacks];
+#pragma unroll
+    for (int i = 0; i < kMaxPacks; ++i) {
+      const int p = tid + kThreads * i;
+      v[i] = (p < npk) ? ld_stream_16(yt + static_cast<size_t>(k) * H + p * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxPacks; ++i) {
+      float f[8];
+      unpack8(v[i], f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(wk, f[j], acc[i][j]);
+    }
+  }
+
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kMaxPacks; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss = fmaf(acc[i][j], acc[i][j], ss);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  __shared__ float part[kThreads / 32];
+  if ((tid & 31) == 0) part[tid >> 5] = ss;
+  __syncthreads();
+  float total = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) total += part[w];
+  const float inv = 1.0f / sqrtf(total / static_cast<float>(H) + eps);
+
+#pragma unroll
+  for (int i = 0; i < kMaxPacks; ++i) {
+    const int p = tid + kThreads * i;
+    if (p >= npk) continue;
+    float g[8];
+    unpack8(*reinterpret_cast<const uint4*>(gamma + p * 8), g);
+    uint4 o, r;
+    o.x = pack_bf16x2(acc[i][0] * inv * g[0], acc[i][1] * inv * g[1]);
+    o.y = pack_bf16x2(acc[i][2] * inv * g[2], acc[i][3] * inv * g[3]);
+    o.z = pack_bf16x2(acc[i][4] * inv * g[4], acc[i][5] * inv * g[5]);
+    o.w = pack_bf16x2(acc[i][6] * inv * g[6], acc[i][7] * inv * g[7]);
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H + p * 8) = o;
+    if (residual_out != nullptr) {
+      r.x = pack_bf16x2(acc[i][0], acc[i][1]);
+      r.y = pack_bf16x2(acc[i][2], acc[i][3]);
+      r.z = pack_bf16x2(acc[i][4], acc[i][5]);
+      r.w = pack_bf16x2(acc[i][6], acc[i][7]);
+      *reinterpret_cast<uint4*>(residual_out + static_cast<size_t>(t) * H + p * 8) = r;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_finalize(const uint16_t* x, const uint16_t* y, const float* topk_w, const uint16_t* gamma,
+                            float eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out,
+                            cudaStream_t stream) {
+  finalize_kernel<<<M, kThreads, 0, stream>>>(x, y, topk_w, gamma, eps, K, H, out, residual_out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

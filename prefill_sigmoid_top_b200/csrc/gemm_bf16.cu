@@ -1,0 +1,328 @@
+// Grouped expert projections on the 5th-generation tensor cores (tcgen05 +
+// tensor memory), fed by TMA, over the expert-major plan
+// ("[flashinfer] ... AlphaMoE NVFP4 커널 최적화", flashinfer PR #6511 analysis:
+// §3-§4 the up kernels, §1-§2 the down kernels, §6 the route chain
+// up -> down -> finalize over the plan of §5).
+//
+// Orientation ("swap AB"): the weight rows are the MMA's M side (128 rows of
+// one expert's W per CTA) and the routed tokens are its N side, so one CTA
+// streams a 128 x K panel of weights through shared memory once and applies
+// it to every token of its tile.  For decode-sized problems the token side is
+// 16..32 wide and the kernel is a weight stream at HBM speed; for prefill the
+// token side grows to 128 and the same kernel becomes a dense contraction.
+//
+// Work unit = (token tile, weight tile).  Token tiles are consecutive plan
+// rows of one expert, at most NMAX wide: expert e owns ceil(count[e]/NMAX)
+// tiles over its real rows (padding rows of the plan are never computed; the
+// MMA width N is the tile's row count rounded up to 16, which stays inside
+// the expert's padded segment because the block size is a multiple of 16).
+// grid.x = weight tiles (fastest, so CTAs launched together share the token
+// tile in L2), grid.y = an upper bound on the token tiles computed on the host
+// without reading the plan back; CTAs past the real count exit at once.
+//
+// Roles in a 128-thread CTA:
+//   warp 0       TMA producer: waits for a free stage, posts the expected
+//                bytes, loads the weight tile(s) (one 128x64 bf16 box each) and
+//                the token rows: up = x rows gathered by token id with
+//                tile::gather4 (4 rows per copy), down = h rows (contiguous
+//                plan rows, 16-row boxes).
+//   warp 1 / t0  MMA issuer: 4 tcgen05.mma (K = 16 each) per 64-wide stage,
+//                per accumulator; tcgen05.commit frees the stage.
+//   warps 0-3    epilogue: tcgen05.ld of the fp32 accumulators (warp w owns
+//                tensor-memory lanes 32w..32w+31 = weight rows), then
+//                up:   h[row, i] = bf16(silu(gate) * up)   (fused SwiGLU)
+//                down: y[slot, j] = bf16(acc), scattered to the slot id.
+// Every wait is bounded; a timeout sets the error word and unwinds.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;        // weight rows per CTA (MMA M)
+constexpr int kBK = 64;         // contraction elements per stage = one 128-byte swizzle row
+constexpr int kATile = kBM * kBK * 2;
+
+constexpr int pow2_at_least(int v) {
+  int p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <bool kUp, int kNmax, int kStages>
+struct Cfg {
+  static constexpr int kBTile = kNmax * kBK * 2;
+  static constexpr int kAPerStage = kUp ? 2 : 1;
+  static constexpr int kStageBytes = kATile * kAPerStage + kBTile;
+  static constexpr int kTmemCols = pow2_at_least(kUp ? 2 * kNmax : kNmax);
+  static constexpr int kMiscBytes = 1024;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMiscBytes;
+  static_assert(kBTile % 1024 == 0, "token tile must keep 1024-byte alignment");
+  static_assert(kNmax % 16 == 0 && kNmax <= 256, "MMA N limits");
+  static_assert(kTmemCols <= 256, "two CTAs per SM share the 512 tensor-memory columns");
+};
+
+template <bool kUp, int kNmax, int kStages>
+__global__ void __launch_bounds__(128, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
+                        const __grid_constant__ CUtensorMap tm_b, const GroupedGemmArgs args) {
+  using C = Cfg<kUp, kNmax, kStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* misc = smem + kStages * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + kStages;
+  uint64_t* accf = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* info = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 1));  // [0] expert, [1] local tile
+  int* tok = info + 2;                                                           // [kNmax]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wt = blockIdx.x;
+  const int tile = blockIdx.y;
+  const int E = args.E;
+
+  // ---- which expert / which of its tiles is token tile `tile`
+  int* cnt = reinterpret_cast<int*>(stages);  // scratch before the pipeline starts (E <= 1024)
+  for (int e = tid; e < E; e += 128) cnt[e] = args.expert_counts[e];
+  if (tid == 0) {
+    info[0] = -1;
+    info[1] = 0;
+    *abort_flag = 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int lo = min(E, lane * per), hi = min(E, lo + per);
+    int sum = 0;
+    for (int e = lo; e < hi; ++e) sum += (cnt[e] + kNmax - 1) / kNmax;
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const int excl = incl - sum;
+    if (tile >= excl && tile < incl) {
+      int t = excl;
+      for (int e = lo; e < hi; ++e) {
+        const int n = (cnt[e] + kNmax - 1) / kNmax;
+        if (tile < t + n) {
+          info[0] = e;
+          info[1] = tile - t;
+          break;
+        }
+        t += n;
+      }
+    }
+  }
+  __syncthreads();
+  const int e = info[0];
+  if (e < 0) return;  // past the real tile count: the whole CTA leaves before any async work
+  const int local = info[1];
+  const int nrows = min(kNmax, cnt[e] - local * kNmax);
+  const int row0 = args.expert_offsets[e] + local * kNmax;
+  const int N = (nrows + 15) & ~15;
+  const int nslots = args.M * args.top_k;
+  for (int n = tid; n < N; n += 128) {
+    int v = kUp ? 0 : -1;
+    if (n < nrows) {
+      const int id = args.sorted_ids[row0 + n];
+      if (id >= 0 && id < nslots) {
+        v = kUp ? id / args.top_k : id;
+      } else {
+        set_error(args.err, kErrInvalidInput);
+      }
+    }
+    tok[n] = v;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();  // also retires the use of `cnt` before TMA writes the stages
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  const int nk = args.kdim / kBK;
+  const int a_row = e * args.rows_per_expert + wt * kBM;
+  const uint32_t b_bytes = static_cast<uint32_t>(N) * kBK * 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensor_map(&tm_a0);
+      if (kUp) prefetch_tensor_map(&tm_a1);
+      prefetch_tensor_map(&tm_b);
+    }
+    const uint64_t pol_w = l2_policy_evict_first();
+    int issued = 0;
+    for (int k = 0; k < nk; ++k) {
+      const int s = k % kStages;
+      const uint32_t ph = (k / kStages) & 1;
+      bool free_slot = true;
+      if (lane == 0) free_slot = mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag);
+      free_slot = __shfl_sync(0xffffffffu, free_slot, 0);  // one decision for the whole warp
+      if (!free_slot) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          set_error(args.err, kErrTimeout);
+        }
+        break;
+      }
+      uint8_t* st = stages + s * C::kStageBytes;
+      uint8_t* bt = st + kATile * C::kAPerStage;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], kATile * C::kAPerStage + b_bytes);
+        tma_load_2d_hint(&tm_a0, &full[s], st, k * kBK, a_row, pol_w);
+        if (kUp) tma_load_2d_hint(&tm_a1, &full[s], st + kATile, k * kBK, a_row, pol_w);
+      }
+      __syncwarp();
+      if (kUp) {
+        for (int i = lane; i < N / 4; i += 32)
+          tma_gather4(&tm_b, &full[s], bt + i * 4 * (kBK * 2), k * kBK, tok[4 * i], tok[4 * i + 1], tok[4 * i + 2],
+                      tok[4 * i + 3]);
+      } else {
+        for (int i = lane; i < N / 16; i += 32)
+          tma_load_2d(&tm_b, &full[s], bt + i * 16 * (kBK * 2), k * kBK, row0 + 16 * i);
+      }
+      issued = k + 1;
+    }
+    // Do not leave while copies issued by this CTA may still land.
+    if (lane == 0) {
+      for (int k = max(0, issued - kStages); k < issued; ++k) {
+        const int s = k % kStages;
+        if (!mbar_wait_bounded(&full[s], (k / kStages) & 1, nullptr)) {
+          set_error(args.err, kErrTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kBM, N);
+      for (int k = 0; k < nk; ++k) {
+        const int s = k % kStages;
+        const uint32_t ph = (k / kStages) & 1;
+        if (!mbar_wait_bounded(&full[s], ph, abort_flag)) {
+          *abort_flag = 1;
+          set_error(args.err, kErrTimeout);
+          break;
+        }
+        tc_fence_after_sync();
+        uint8_t* st = stages + s * C::kStageBytes;
+        const uint64_t da0 = umma_desc_sw128(st);
+        const uint64_t db = umma_desc_sw128(st + kATile * C::kAPerStage);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint32_t acc = (k | kk) != 0 ? 1u : 0u;
+          umma_bf16_ss(tmem, da0 + 2 * kk, db + 2 * kk, idesc, acc);
+          if (kUp) {
+            const uint64_t da1 = umma_desc_sw128(st + kATile);
+            umma_bf16_ss(tmem + kNmax, da1 + 2 * kk, db + 2 * kk, idesc, acc);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+    }
+    __syncwarp();
+  }
+
+  // ---------------------------------------------------- epilogue (all warps)
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait_bounded(accf, 0, nullptr);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  tc_fence_after_sync();
+  if (!ok && lane == 0) set_error(args.err, kErrTimeout);
+  const bool go = __shfl_sync(0xffffffffu, ok && !*abort_flag, 0);
+  if (go) {
+    const int wrow = wt * kBM + warp * 32 + lane;  // output column: I index (up) or H index (down)
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int c = 0; c < N; c += 16) {
+      uint32_t d0[16];
+      tmem_load_16(lane_base + c, d0);
+      if (kUp) {
+        uint32_t d1[16];
+        tmem_load_16(lane_base + kNmax + c, d1);
+        tmem_load_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int n = c + q;
+          if (n < nrows) {
+            const float g = __uint_as_float(d0[q]);
+            const float u = __uint_as_float(d1[q]);
+            const float hv = g / (1.0f + expf(-g)) * u;
+            reinterpret_cast<__nv_bfloat16*>(args.out)[static_cast<size_t>(row0 + n) * args.out_ld + wrow] =
+                __float2bfloat16_rn(hv);
+          }
+        }
+      } else {
+        tmem_load_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int n = c + q;
+          if (n < nrows) {
+            const int slot = tok[n];
+            if (slot >= 0)
+              reinterpret_cast<__nv_bfloat16*>(args.out)[static_cast<size_t>(slot) * args.out_ld + wrow] =
+                  __float2bfloat16_rn(__uint_as_float(d0[q]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+template <bool kUp, int kNmax, int kStages>
+cudaError_t launch_variant(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                           const GroupedGemmArgs& args, cudaStream_t stream) {
+  using C = Cfg<kUp, kNmax, kStages>;
+  auto kern = grouped_gemm_kernel<kUp, kNmax, kStages>;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  static bool done[64] = {};
+  if (dev < 64 && !done[dev]) {
+    st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (st != cudaSuccess) return st;
+    done[dev] = true;
+  }
+  const long long mk = static_cast<long long>(args.M) * args.top_k;
+  const long long tiles_ub = mk / kNmax + (mk < args.E ? mk : args.E);
+  dim3 grid(args.rows_per_expert / kBM, static_cast<unsigned>(tiles_ub));
+  kern<<<grid, 128, C::kSmemBytes, stream>>>(a0, a1, b, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                              const GroupedGemmArgs& args, int nmax, cudaStream_t stream) {
+  if (nmax <= 32) return launch_variant<true, 32, 3>(w_gate, w_up, x_rows, args, stream);
+  return launch_variant<true, 128, 2>(w_gate, w_up, x_rows, args, stream);
+}
+
+cudaError_t launch_grouped_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
+                                int nmax, cudaStream_t stream) {
+  if (nmax <= 32) return launch_variant<false, 32, 5>(w_down, w_down, h_rows, args, stream);
+  return launch_variant<false, 128, 3>(w_down, w_down, h_rows, args, stream);
+}
+
+}  // namespace moe

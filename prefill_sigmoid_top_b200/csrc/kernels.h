@@ -1,0 +1,48 @@
+// Internal launchers shared between the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// router.cu
+cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
+                                 float* logits, cudaStream_t stream);
+cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t* topk_ids, float* topk_w,
+                               cudaStream_t stream);
+
+// align.cu
+cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, int32_t* sorted_ids,
+                         int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets, int32_t* ntpp,
+                         int32_t* err, cudaStream_t stream);
+
+// finalize.cu
+cudaError_t launch_finalize(const uint16_t* x, const uint16_t* y, const float* topk_w, const uint16_t* gamma,
+                            float eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out,
+                            cudaStream_t stream);
+
+// gemm_bf16.cu: grouped projections over the expert-major plan.
+struct GroupedGemmArgs {
+  const int32_t* sorted_ids;
+  const int32_t* expert_counts;
+  const int32_t* expert_offsets;
+  uint16_t* out;       // up: h [cap, I]; down: y [M*K, H]
+  int32_t* err;        // device error word (nullable)
+  int M, E, top_k;
+  int rows_per_expert; // up: I; down: H  (weight rows of one expert)
+  int kdim;            // up: H; down: I  (contraction length)
+  int out_ld;          // up: I; down: H
+};
+
+// `nmax` selects the token-tile width (32 or 128).  Tensor maps: a0/a1 are
+// the weight matrices viewed as 2-D [E*rows_per_expert, kdim]; b is x [M,H]
+// (up, row gather) or h [cap, I] (down, contiguous rows).
+cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                              const GroupedGemmArgs& args, int nmax, cudaStream_t stream);
+cudaError_t launch_grouped_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
+                                int nmax, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,176 @@
+// Sigmoid top-k router ("[sglang] [NPU] GLM-4.7-Flash 성능 최적화", sglang
+// PR #29509 analysis, §2 "MoE TopK Scoring Function": scores are sigmoid,
+// norm_type=1, rather than softmax).
+//
+// Two launches:
+//  1. router_logits_kernel: z[t,e] = x[t] . w_router[e] + bias[e] in fp32, in
+//     the canonical order that makes the selection reproducible bit for bit:
+//     lane l of a warp accumulates, one fma per element and in increasing h,
+//     the elements h = 256*j + 8*l + i (i = 0..7, j = 0..H/256-1), i.e. the
+//     16-byte chunk the lane loads in a coalesced 512-byte warp load; the 32
+//     lane partials are then combined with an xor butterfly (offsets 16, 8, 4,
+//     2, 1), which adds partial l and l+16 first, then the results 8 apart,
+//     and so on; the bias is added last.
+//     Register tiling: each lane carries 8 tokens x 4 experts partials, so a
+//     chunk of x and of w_router is loaded once per 32 fmas.
+//  2. router_topk_kernel: one warp per token selects the K largest logits
+//     (descending; equal logits -> lower expert id) by K rounds of a warp
+//     argmax, then w_k = s_k / sum s with s = 1 / (1 + exp(-z)).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kTokPerWarp = 8;
+constexpr int kExpPerWarp = 4;
+constexpr int kWarps = 4;
+
+__device__ __forceinline__ uint4 ld_nc_16(const uint16_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float elem(const uint4& v, int i) {
+  const uint32_t w = (i < 2) ? v.x : (i < 4) ? v.y : (i < 6) ? v.z : v.w;
+  return (i & 1) ? bf16_hi(w) : bf16_lo(w);
+}
+
+__global__ void __launch_bounds__(kWarps * 32) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                                    const uint16_t* __restrict__ w_router,
+                                                                    const float* __restrict__ bias, int M, int H,
+                                                                    int E, float* __restrict__ logits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kTokPerWarp;
+  const int e0 = (blockIdx.y * kWarps + warp) * kExpPerWarp;
+  if (e0 >= E) return;
+
+  float acc[kTokPerWarp][kExpPerWarp];
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+    for (int q = 0; q < kExpPerWarp; ++q) acc[t][q] = 0.0f;
+
+  const int nchunk = H / 256;
+#pragma unroll 1
+  for (int j = 0; j < nchunk; ++j) {
+    const int h = 256 * j + 8 * lane;
+    uint4 wv[kExpPerWarp], xv[kTokPerWarp];
+#pragma unroll
+    for (int q = 0; q < kExpPerWarp; ++q)
+      wv[q] = (e0 + q < E) ? ld_nc_16(w_router + static_cast<size_t>(e0 + q) * H + h) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int t = 0; t < kTokPerWarp; ++t)
+      xv[t] = (t0 + t < M) ? ld_nc_16(x + static_cast<size_t>(t0 + t) * H + h) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)  // increasing h inside the chunk
+#pragma unroll
+      for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+        for (int q = 0; q < kExpPerWarp; ++q) acc[t][q] = __fmaf_rn(elem(xv[t], i), elem(wv[q], i), acc[t][q]);
+  }
+
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+    for (int q = 0; q < kExpPerWarp; ++q) {
+      float v = acc[t][q];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+      acc[t][q] = v;
+    }
+  // lane l stores pair l = (t, q) = (l / 4, l % 4)
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+    for (int q = 0; q < kExpPerWarp; ++q)
+      if (lane == t * kExpPerWarp + q && t0 + t < M && e0 + q < E) {
+        const float b = bias != nullptr ? bias[e0 + q] : 0.0f;
+        logits[static_cast<size_t>(t0 + t) * E + e0 + q] = __fadd_rn(acc[t][q], b);
+      }
+}
+
+// (value, id) ordering of the selection: larger value first, then lower id.
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+template <int kPerLane>
+__global__ void __launch_bounds__(128) router_topk_kernel(const float* __restrict__ logits, int M, int E, int K,
+                                                          int32_t* __restrict__ topk_ids,
+                                                          float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (t >= M) return;
+  float v[kPerLane];
+  bool live[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int e = lane + 32 * i;
+    live[i] = e < E;
+    v[i] = live[i] ? logits[static_cast<size_t>(t) * E + e] : -INFINITY;
+  }
+  float sel_v = 0.0f;
+  int sel_id = 0;
+  for (int k = 0; k < K; ++k) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)
+      if (live[i] && better(v[i], lane + 32 * i, bv, bi)) {
+        bv = v[i];
+        bi = lane + 32 * i;
+      }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)  // the owner retires the winner
+      if (lane + 32 * i == bi) live[i] = false;
+    if (lane == k) {
+      sel_v = bv;
+      sel_id = bi;
+    }
+  }
+  const float s = (lane < K) ? 1.0f / (1.0f + expf(-sel_v)) : 0.0f;
+  float total = s;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+  if (lane < K) {
+    topk_ids[static_cast<size_t>(t) * K + lane] = sel_id;
+    topk_w[static_cast<size_t>(t) * K + lane] = s / total;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
+                                 float* logits, cudaStream_t stream) {
+  const int experts_per_block = kWarps * kExpPerWarp;
+  dim3 grid((M + kTokPerWarp - 1) / kTokPerWarp, (E + experts_per_block - 1) / experts_per_block);
+  router_logits_kernel<<<grid, kWarps * 32, 0, stream>>>(x, w_router, bias, M, H, E, logits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t* topk_ids, float* topk_w,
+                               cudaStream_t stream) {
+  dim3 grid((M + 3) / 4);
+  if (E <= 64)
+    router_topk_kernel<2><<<grid, 128, 0, stream>>>(logits, M, E, K, topk_ids, topk_w);
+  else if (E <= 256)
+    router_topk_kernel<8><<<grid, 128, 0, stream>>>(logits, M, E, K, topk_ids, topk_w);
+  else
+    router_topk_kernel<32><<<grid, 128, 0, stream>>>(logits, M, E, K, topk_ids, topk_w);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,108 @@
+"""The C-ABI library: loads, exports every symbol the header declares, validates on the host.
+
+No compute call is made here: every call below fails host validation before
+any CUDA work, so these tests run without a GPU (and launch nothing with one).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import prefill_sigmoid_top_b200 as moe
+from prefill_sigmoid_top_b200 import _Plan, _Shape, _Weights, _Layout
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+FAKE = ctypes.c_void_p(0x10000)       # aligned non-null address, never dereferenced
+FAKE_MIS = ctypes.c_void_p(0x10008)   # 8-byte aligned only
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 15
+    L = moe.library()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for code, name in moe.STATUS.items():
+        assert moe.status_string(code).startswith(name)
+
+
+C0 = moe.Shape(M=16, H=256, I=128, E=8, top_k=2, block_size=16)
+C1 = moe.Shape(M=8, H=7168, I=2048, E=256, top_k=16, block_size=16)
+
+
+def test_sizes():
+    assert moe.align_capacity(C0) == 16 * 2 + 8 * 15
+    assert moe.align_capacity(C1) == 8 * 16 + 256 * 15
+    assert moe.route_workspace_size(C1) >= 8 * 256 * 4
+    lay = moe.layer_workspace_layout(C1)
+    assert lay["total"] == moe.layer_workspace_size(C1)
+    offs = [lay[k] for k in ["err_flag", "logits", "topk_ids", "topk_w", "sorted_ids", "block_expert",
+                             "expert_counts", "expert_offsets", "num_tokens_post_padded", "h", "y"]]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lay["y"] - lay["h"] >= moe.align_capacity(C1) * 2048 * 2
+    assert lay["total"] - lay["y"] >= 8 * 16 * 7168 * 2
+
+
+@pytest.mark.parametrize("bad", [
+    dict(H=255), dict(H=8448), dict(I=64), dict(E=0), dict(E=1025), dict(top_k=0), dict(top_k=9),
+    dict(block_size=24), dict(block_size=8), dict(block_size=512), dict(M=0),
+])
+def test_unsupported_shapes(bad):
+    kw = dict(M=16, H=256, I=128, E=8, top_k=2, block_size=16)
+    kw.update(bad)
+    s = moe.Shape(**kw)
+    assert moe.align_capacity(s) == 0
+    L = moe.library()
+    st = L.moe_route(FAKE, FAKE, None, s.c(), FAKE, FAKE, FAKE, 1 << 20, None)
+    assert st == 2
+
+
+def test_null_and_misaligned_pointers():
+    L = moe.library()
+    s = C0.c()
+    assert L.moe_route(None, FAKE, None, s, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.moe_route(FAKE_MIS, FAKE, None, s, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.moe_route(FAKE, FAKE, None, s, FAKE, FAKE, None, 0, None) == 3   # no workspace
+    assert L.moe_route(FAKE, FAKE, None, s, FAKE, FAKE, FAKE, 4, None) == 3   # too small
+    assert L.moe_align_block_size(FAKE, s, None, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert L.moe_finalize_rmsnorm(FAKE, FAKE, FAKE, FAKE, ctypes.c_float(1e-5), s, None, None, None) == 1
+    assert L.moe_finalize_rmsnorm(FAKE, FAKE, FAKE, FAKE, ctypes.c_float(-1.0), s, FAKE, None, None) == 1
+    w = _Weights(0, 0x10000, 0x10000, 0x10000, None, None, None)
+    p = _Plan(0x10000, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert L.moe_grouped_up_swiglu(None, ctypes.byref(w), ctypes.byref(p), s, FAKE, None, 0, None, None) == 1
+    assert L.moe_grouped_up_swiglu(FAKE, None, ctypes.byref(p), s, FAKE, None, 0, None, None) == 1
+    assert L.moe_grouped_up_swiglu(FAKE, ctypes.byref(w), None, s, FAKE, None, 0, None, None) == 1
+    assert L.moe_grouped_down(FAKE, ctypes.byref(w), ctypes.byref(p), s, FAKE_MIS, None, 0, None, None) == 1
+    w_nv = _Weights(7, 0x10000, 0x10000, 0x10000, None, None, None)
+    assert L.moe_grouped_down(FAKE, ctypes.byref(w_nv), ctypes.byref(p), s, FAKE, None, 0, None, None) == 2
+
+
+def test_layer_workspace_checks():
+    L = moe.library()
+    s = C0.c()
+    w = _Weights(0, 0x10000, 0x10000, 0x10000, None, None, None)
+    need = moe.layer_workspace_size(C0)
+    args = [FAKE, FAKE, None, ctypes.byref(w), FAKE, ctypes.c_float(1e-5), s, FAKE, None, None, None]
+    assert L.moe_layer(*args, None, need, None) == 3
+    assert L.moe_layer(*args, FAKE, need - 1, None) == 3
+    assert L.moe_layer(FAKE, FAKE, None, None, FAKE, ctypes.c_float(1e-5), s, FAKE, None, None, None, FAKE, need,
+                       None) == 1
+    lay = _Layout()
+    assert L.moe_layer_workspace_layout(s, 0, None) == 1
+    assert L.moe_layer_workspace_layout(s, 0, ctypes.byref(lay)) == 0 and lay.total == need
+
+
+def test_device_error_rejects_null():
+    code = ctypes.c_int32(0)
+    assert moe.library().moe_get_device_error(None, None, ctypes.byref(code)) == 1

@@ -1,0 +1,373 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars: routing ids, slot order and the whole plan bit-exact; routing weights
+within 1e-6; the layer output within 2e-2 x RMS(oracle output) (bf16).
+Intermediates h and y (diagnostics) elementwise within 2^-7 |ref| + 1e-2 RMS(ref).
+Outputs are poisoned (0xFF bytes: NaN for bf16/fp32, -1 for int32) before each
+call and guarded by canary bytes after the buffer.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import prefill_sigmoid_top_b200 as moe
+from prefill_sigmoid_top_b200 import inputs
+from tests._util import bf16_bits, bits_to_f64, rms
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+CANARY = 0x5A
+
+
+def guarded(n, dtype, device=DEV):
+    """A poisoned tensor of n elements followed by 256 canary bytes in the same allocation."""
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    raw = torch.full((nbytes + 256,), 0xFF, dtype=torch.uint8, device=device)
+    raw[nbytes:] = CANARY
+    return raw, raw[:nbytes].view(dtype)
+
+
+def canary_ok(raw, n, dtype):
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    return bool((raw[nbytes:] == CANARY).all().item())
+
+
+def close_elementwise(got, ref, rel=2.0 ** -7, abs_rms=1e-2):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    tol = rel * np.abs(ref) + abs_rms * rms(ref)
+    bad = np.abs(got - ref) > tol
+    return (not bad.any()), float(np.abs(got - ref).max()), int(bad.sum())
+
+
+def to_dev(cfg, dev=DEV):
+    return inputs.make_inputs(cfg, dev)
+
+
+def host_bits(d):
+    return dict(x=bf16_bits(d["x"]), w_router=bf16_bits(d["w_router"]), bias=d["bias"].cpu().numpy(),
+                gamma=bf16_bits(d["gamma"]))
+
+
+def expert_lists(d, experts, E):
+    wg, wu, wd = [None] * E, [None] * E, [None] * E
+    for e in sorted(set(int(v) for v in experts)):
+        wg[e] = bf16_bits(d["w_gate"][e])
+        wu[e] = bf16_bits(d["w_up"][e])
+        wd[e] = bf16_bits(d["w_down"][e])
+    return wg, wu, wd
+
+
+SMALL_ROUTER_SHAPES = [
+    # M, H, E, K, bias
+    (16, 256, 8, 2, "zero"), (1, 256, 8, 2, "normal"), (3, 512, 33, 5, "normal"), (37, 1024, 64, 8, "normal"),
+    (100, 256, 256, 16, "normal"), (17, 768, 1, 1, "normal"), (9, 256, 1000, 32, "normal"), (64, 2048, 128, 4, "zipf"),
+]
+
+
+@pytest.mark.parametrize("M,H,E,K,bias", SMALL_ROUTER_SHAPES)
+def test_router_bitexact_small(M, H, E, K, bias):
+    cfg = inputs.CONFIGS[0].with_(M=M, H=H, E=E, K=K, bias=bias, seed=M * 7 + E)
+    w_r, b, g, x = inputs.router_inputs(cfg)
+    ids, w = moe.route(x.to(DEV), w_r.to(DEV), b.to(DEV), K)
+    ids_o, w_o = oracle.route(bf16_bits(x), bf16_bits(w_r), b.numpy(), K)
+    assert np.array_equal(ids.cpu().numpy(), ids_o)
+    assert np.abs(w.cpu().numpy() - w_o).max() <= 1e-6
+
+
+def test_router_ties_exact():
+    # every logit equal (zero router weights, zero bias): ids must be 0..K-1
+    M, H, E, K = 5, 256, 16, 4
+    x = torch.randn(M, H).to(torch.bfloat16).to(DEV)
+    w_r = torch.zeros(E, H, dtype=torch.bfloat16, device=DEV)
+    ids, w = moe.route(x, w_r, None, K)
+    assert (ids.cpu() == torch.arange(K, dtype=torch.int32).expand(M, K)).all()
+    assert torch.allclose(w.cpu(), torch.full((M, K), 1.0 / K), atol=1e-7)
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4])
+def test_router_bitexact_full_size(cid):
+    cfg = inputs.CONFIGS[cid]
+    w_r, b, g, x = inputs.router_inputs(cfg)
+    ids, w = moe.route(x.to(DEV), w_r.to(DEV), b.to(DEV), cfg.K)
+    ids_o, w_o = oracle.route(bf16_bits(x), bf16_bits(w_r), b.numpy(), cfg.K)
+    assert np.array_equal(ids.cpu().numpy(), ids_o)
+    assert np.abs(w.cpu().numpy() - w_o).max() <= 1e-6
+
+
+# ------------------------------------------------------------------ align
+def _gpu_plan(ids_np, E, B, err=None):
+    M, K = ids_np.shape
+    shape = moe.Shape(M, 256, 128, E, K, B)
+    cap = moe.align_capacity(shape)
+    raws = {}
+    out = {}
+    for name, n in [("sorted_ids", cap), ("block_expert", cap // B + 1), ("expert_counts", E),
+                    ("expert_offsets", E + 1), ("num_tokens_post_padded", 1)]:
+        raws[name], out[name] = guarded(n, torch.int32)
+    ids = torch.from_numpy(np.ascontiguousarray(ids_np, np.int32)).to(DEV)
+    moe.align_block_size(ids, E, B, err_flag=err, out=out)
+    torch.cuda.synchronize()
+    for name, n in [("sorted_ids", cap), ("block_expert", cap // B + 1), ("expert_counts", E),
+                    ("expert_offsets", E + 1), ("num_tokens_post_padded", 1)]:
+        assert canary_ok(raws[name], n, torch.int32), name
+    return {k: v.cpu().numpy() for k, v in out.items()}
+
+
+def _compare_plan(g, o, B):
+    n = o["ntpp"]
+    assert int(g["num_tokens_post_padded"][0]) == n
+    assert np.array_equal(g["expert_counts"], o["counts"])
+    assert np.array_equal(g["expert_offsets"], o["offsets"])
+    assert np.array_equal(g["sorted_ids"][:n], o["sorted_ids"])
+    assert np.array_equal(g["block_expert"][: n // B], o["block_expert"])
+
+
+ALIGN_CASES = [(16, 2, 8, 16), (8, 16, 256, 16), (512, 16, 256, 64), (2048, 16, 256, 128), (1000, 16, 256, 16),
+               (1, 1, 1, 16), (37, 5, 64, 32), (300, 8, 1024, 256), (5, 3, 3, 128), (4096, 8, 16, 16)]
+
+
+@pytest.mark.parametrize("M,K,E,B", ALIGN_CASES)
+def test_align_bitexact(M, K, E, B):
+    rng = np.random.default_rng(M + 3 * E + B)
+    ids = np.stack([rng.choice(E, size=K, replace=False) for _ in range(M)]).astype(np.int32)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    g = _gpu_plan(ids, E, B, err)
+    assert moe.get_device_error(err) == 0
+    _compare_plan(g, oracle.align(ids, E, B), B)
+
+
+def test_align_skewed_and_empty():
+    rng = np.random.default_rng(77)
+    E, K, M, B = 256, 16, 2048, 128
+    p = 1.0 / np.arange(1, E + 1) ** 1.1
+    p[200:] = 0.0
+    ids = np.stack([rng.choice(E, size=K, replace=False, p=p / p.sum()) for _ in range(M)]).astype(np.int32)
+    g = _gpu_plan(ids, E, B)
+    _compare_plan(g, oracle.align(ids, E, B), B)
+
+
+@pytest.mark.parametrize("bad", [-1, 8, 1 << 20])
+def test_align_invalid_id_sets_error_without_fault(bad):
+    ids = np.array([[0, 1], [2, bad], [3, 4]], np.int32)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    _gpu_plan(ids, 8, 16, err)
+    assert moe.get_device_error(err) == 4  # MOE_ERR_INVALID_INPUT
+    # the library stays usable afterwards
+    ids_ok = np.array([[0, 1], [2, 3]], np.int32)
+    _compare_plan(_gpu_plan(ids_ok, 8, 16), oracle.align(ids_ok, 8, 16), 16)
+
+
+def test_align_repeat_stress():
+    # many calls on fresh random inputs; every result bit-exact against the oracle
+    rng = np.random.default_rng(2024)
+    for it in range(300):
+        E = int(rng.choice([8, 64, 256, 1024]))
+        K = int(rng.integers(1, min(E, 16) + 1))
+        M = int(rng.integers(1, 600))
+        B = int(rng.choice([16, 32, 64, 128, 256]))
+        ids = rng.integers(0, E, size=(M, K)).astype(np.int32)
+        _compare_plan(_gpu_plan(ids, E, B), oracle.align(ids, E, B), B)
+
+
+def test_align_repeat_deterministic():
+    rng = np.random.default_rng(5)
+    ids = torch.from_numpy(rng.integers(0, 256, size=(2048, 16)).astype(np.int32)).to(DEV)
+    first = moe.align_block_size(ids, 256, 128)
+    ref = {k: v.clone() for k, v in first.items()}
+    n = int(ref["num_tokens_post_padded"].item())
+    for _ in range(2000):
+        out = moe.align_block_size(ids, 256, 128, out=first)
+    torch.cuda.synchronize()
+    assert torch.equal(out["sorted_ids"][:n], ref["sorted_ids"][:n])
+    assert torch.equal(out["block_expert"][: n // 128], ref["block_expert"][: n // 128])
+
+
+# ------------------------------------------------------------------ finalize
+@pytest.mark.parametrize("M,K,H", [(1, 1, 256), (16, 2, 256), (7, 16, 7168), (33, 4, 8192), (5, 3, 1280)])
+def test_finalize(M, K, H):
+    gen = torch.Generator().manual_seed(M * K + H)
+    x = torch.randn(M, H, generator=gen).to(torch.bfloat16)
+    y = torch.randn(M, K, H, generator=gen).to(torch.bfloat16)
+    w = torch.softmax(torch.randn(M, K, generator=gen), dim=1).float()
+    gamma = (1 + 0.1 * torch.randn(H, generator=gen)).to(torch.bfloat16)
+    raw_o, out = guarded(M * H, torch.bfloat16)
+    raw_r, res = guarded(M * H, torch.bfloat16)
+    moe.finalize_rmsnorm(x.to(DEV), y.to(DEV), w.to(DEV), gamma.to(DEV), 1e-5, out=out.view(M, H),
+                         residual_out=res.view(M, H), want_residual=True)
+    torch.cuda.synchronize()
+    assert canary_ok(raw_o, M * H, torch.bfloat16) and canary_ok(raw_r, M * H, torch.bfloat16)
+    o_out, o_res = oracle.finalize(bf16_bits(x), bf16_bits(y), w.double().numpy(), bf16_bits(gamma), 1e-5)
+    ok, err, nbad = close_elementwise(bits_to_f64(bf16_bits(out.view(M, H))), bits_to_f64(o_out), abs_rms=1e-3)
+    assert ok, (err, nbad)
+    ok, err, nbad = close_elementwise(bits_to_f64(bf16_bits(res.view(M, H))), bits_to_f64(o_res), abs_rms=1e-3)
+    assert ok, (err, nbad)
+
+
+# ------------------------------------------------------------------ grouped projections
+GEMM_CASES = [
+    # cfg overrides (M, H, I, E, K, B)
+    dict(M=16, H=256, I=128, E=8, K=2, B=16),
+    dict(M=40, H=512, I=256, E=16, K=4, B=16),
+    dict(M=300, H=256, I=384, E=8, K=3, B=64),   # many rows per expert: several 128-row tiles + ragged tail
+    dict(M=5, H=1024, I=128, E=64, K=6, B=32),
+]
+
+
+@pytest.mark.parametrize("nmax", ["32", "128"])
+@pytest.mark.parametrize("case", GEMM_CASES)
+def test_grouped_up_down(case, nmax, monkeypatch):
+    monkeypatch.setenv("MOE_GEMM_NMAX", nmax)
+    cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + case["E"], **case)
+    d = to_dev(cfg)
+    hb = host_bits(d)
+    ids_o, w_o = oracle.route(hb["x"], hb["w_router"], hb["bias"], cfg.K)
+    plan_o = oracle.align(ids_o, cfg.E, cfg.B)
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    cap = moe.align_capacity(shape)
+    # the oracle's plan, laid out as the library expects
+    sorted_full = np.full(cap, -1, np.int32)
+    sorted_full[: plan_o["ntpp"]] = plan_o["sorted_ids"]
+    bexp = np.zeros(cap // cfg.B + 1, np.int32)
+    bexp[: len(plan_o["block_expert"])] = plan_o["block_expert"]
+    plan = dict(sorted_ids=torch.from_numpy(sorted_full).to(DEV), block_expert=torch.from_numpy(bexp).to(DEV),
+                expert_counts=torch.from_numpy(plan_o["counts"]).to(DEV),
+                expert_offsets=torch.from_numpy(plan_o["offsets"]).to(DEV),
+                num_tokens_post_padded=torch.tensor([plan_o["ntpp"]], dtype=torch.int32, device=DEV))
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    raw_h, h = guarded(cap * cfg.I, torch.bfloat16)
+    h = h.view(cap, cfg.I)
+    moe.grouped_up_swiglu(d["x"], d["w_gate"], d["w_up"], plan, shape, h=h, err_flag=err)
+    raw_y, y = guarded(cfg.M * cfg.K * cfg.H, torch.bfloat16)
+    y = y.view(cfg.M * cfg.K, cfg.H)
+    moe.grouped_down(h, d["w_down"], plan, shape, y=y, err_flag=err)
+    torch.cuda.synchronize()
+    assert moe.get_device_error(err) == 0
+    assert canary_ok(raw_h, cap * cfg.I, torch.bfloat16) and canary_ok(raw_y, cfg.M * cfg.K * cfg.H, torch.bfloat16)
+    wg, wu, wd = expert_lists(d, range(cfg.E), cfg.E)
+    r = oracle.layer(hb["x"], hb["w_router"], hb["bias"], wg, wu, wd, hb["gamma"], cfg.eps, cfg.K, want_h=True)
+    assert np.array_equal(r["ids"], ids_o)
+    h_np = bits_to_f64(bf16_bits(h))
+    real = plan_o["sorted_ids"] < cfg.M * cfg.K
+    rows = np.nonzero(real)[0]
+    slots = plan_o["sorted_ids"][real]
+    h_ref = bits_to_f64(r["h"].reshape(cfg.M * cfg.K, cfg.I))[slots]
+    ok, e, nbad = close_elementwise(h_np[rows], h_ref)
+    assert ok, ("h", e, nbad)
+    # padding rows are never written: still poisoned
+    pad_rows = np.nonzero(~real)[0]
+    if len(pad_rows):
+        assert np.isnan(h_np[pad_rows]).all()
+    y_ref = bits_to_f64(r["y"].reshape(cfg.M * cfg.K, cfg.H))
+    ok, e, nbad = close_elementwise(bits_to_f64(bf16_bits(y)), y_ref)
+    assert ok, ("y", e, nbad)
+
+
+# ------------------------------------------------------------------ whole layer
+def run_layer(d, cfg, stream_sync=True):
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    ws = torch.empty(moe.layer_workspace_size(shape), dtype=torch.uint8, device=DEV)
+    raw_o, out = guarded(cfg.M * cfg.H, torch.bfloat16)
+    raw_r, res = guarded(cfg.M * cfg.H, torch.bfloat16)
+    ids = torch.full((cfg.M, cfg.K), -1, dtype=torch.int32, device=DEV)
+    tw = torch.full((cfg.M, cfg.K), float("nan"), dtype=torch.float32, device=DEV)
+    moe.layer(d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"], cfg.eps, cfg.K,
+              cfg.B, ws=ws, out=out.view(cfg.M, cfg.H), residual_out=res.view(cfg.M, cfg.H), topk_ids=ids,
+              topk_w=tw)
+    torch.cuda.synchronize()
+    assert canary_ok(raw_o, cfg.M * cfg.H, torch.bfloat16) and canary_ok(raw_r, cfg.M * cfg.H, torch.bfloat16)
+    lay = moe.layer_workspace_layout(shape)
+    err = ws[lay["err_flag"]:lay["err_flag"] + 4].view(torch.int32)
+    assert moe.get_device_error(err) == 0
+    return dict(out=bf16_bits(out.view(cfg.M, cfg.H)), res=bf16_bits(res.view(cfg.M, cfg.H)),
+                ids=ids.cpu().numpy(), w=tw.cpu().numpy(), ws=ws, lay=lay)
+
+
+LAYER_SMALL = [
+    inputs.CONFIGS[0],
+    inputs.CONFIGS[0].with_(M=40, H=512, I=256, E=16, K=4, B=16, seed=11, bias="normal"),
+    inputs.CONFIGS[0].with_(M=257, H=768, I=256, E=32, K=8, B=64, seed=12, bias="zipf"),
+    inputs.CONFIGS[0].with_(M=3, H=256, I=128, E=4, K=4, B=16, seed=13, bias="normal"),
+]
+
+
+@pytest.mark.parametrize("cfg", LAYER_SMALL, ids=lambda c: f"M{c.M}_E{c.E}_K{c.K}")
+def test_layer_small(cfg):
+    d = to_dev(cfg)
+    g = run_layer(d, cfg)
+    hb = host_bits(d)
+    wg, wu, wd = expert_lists(d, range(cfg.E), cfg.E)
+    r = oracle.layer(hb["x"], hb["w_router"], hb["bias"], wg, wu, wd, hb["gamma"], cfg.eps, cfg.K)
+    assert np.array_equal(g["ids"], r["ids"])
+    assert np.abs(g["w"] - r["w"]).max() <= 1e-6
+    ref = bits_to_f64(r["out"])
+    assert np.abs(bits_to_f64(g["out"]) - ref).max() <= 2e-2 * rms(ref)
+    rref = bits_to_f64(r["residual"])
+    assert np.abs(bits_to_f64(g["res"]) - rref).max() <= 2e-2 * rms(rref)
+
+
+def _sample_tokens(ids_o, n_random, seed):
+    """Tokens routed to the busiest expert (first and last) plus random ones."""
+    M, K = ids_o.shape
+    counts = np.bincount(ids_o.ravel(), minlength=int(ids_o.max()) + 1)
+    hot = int(np.argmax(counts))
+    on_hot = np.nonzero((ids_o == hot).any(axis=1))[0]
+    rng = np.random.default_rng(seed)
+    pick = {int(on_hot[0]), int(on_hot[-1])} | set(int(t) for t in rng.choice(M, size=min(M, n_random),
+                                                                               replace=False))
+    return np.array(sorted(pick), np.int32)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cid", [1, 2, 3])
+def test_layer_full_size_sampled(cid):
+    cfg = inputs.CONFIGS[cid]
+    d = to_dev(cfg)
+    g = run_layer(d, cfg)
+    hb = host_bits(d)
+    ids_o, w_o = oracle.route(hb["x"], hb["w_router"], hb["bias"], cfg.K)
+    assert np.array_equal(g["ids"], ids_o)
+    assert np.abs(g["w"] - w_o).max() <= 1e-6
+    tokens = np.arange(cfg.M, dtype=np.int32) if cfg.M <= 8 else _sample_tokens(ids_o, 3, cid)
+    wg, wu, wd = expert_lists(d, ids_o[tokens].ravel(), cfg.E)
+    r = oracle.layer(hb["x"], hb["w_router"], hb["bias"], wg, wu, wd, hb["gamma"], cfg.eps, cfg.K, tokens=tokens)
+    ref = bits_to_f64(r["out"])
+    got = bits_to_f64(g["out"][tokens])
+    assert np.abs(got - ref).max() <= 2e-2 * rms(ref)
+    # diagnostics: y of the sampled slots from the layer's workspace
+    lay = g["lay"]
+    ybytes = cfg.M * cfg.K * cfg.H * 2
+    y = g["ws"][lay["y"]:lay["y"] + ybytes].view(torch.bfloat16).view(cfg.M, cfg.K, cfg.H)
+    y_got = bits_to_f64(bf16_bits(y[torch.from_numpy(tokens).long().to(DEV)]))
+    ok, e, nbad = close_elementwise(y_got, bits_to_f64(r["y"]))
+    assert ok, ("y", e, nbad)
+
+
+def test_layer_cuda_graph_replay():
+    cfg = LAYER_SMALL[1]
+    d = to_dev(cfg)
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    ws = torch.empty(moe.layer_workspace_size(shape), dtype=torch.uint8, device=DEV)
+    out = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.layer(d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"], cfg.eps,
+                  cfg.K, cfg.B, ws=ws, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    eager = out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        moe.layer(d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"], cfg.eps,
+                  cfg.K, cfg.B, ws=ws, out=out)
+    for _ in range(3):
+        out.fill_(float("nan"))     # poison before each replay
+        ws.fill_(0xFF)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    del graph
