@@ -1,0 +1,412 @@
+#!/usr/bin/env python3
+"""Benchmark of the routed-MoE layer on B200 (one JSON line on rank 0).
+
+Default workload: decode, M=8 tokens (H=7168, I=2048, E=256, top_k=16, block 16,
+seed 1).  One step = one pass of the whole layer: route -> align -> up+SwiGLU
+-> down -> finalize+RMSNorm, inputs resident in HBM.  The expert weights are
+22.5 GB and each step streams the touched experts' weights (several GB), far
+more than the 126 MB L2, so no L2 flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+Multi-GPU: the layer is run as independent replicas, one per rank (no
+collective on the data path); rank 0 prints the max-over-ranks time.
+--impl reference times the CPU oracle (fp64 C++) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+# ncu DRAM traffic of the dominant kernel, per launch, measured on the decode
+# workload (profiles/grouped_up_decode_m8.md).  Valid only while the kernel
+# sources hash to KERNEL_HASH; otherwise "traffic" is reported as null.
+NCU_TRAFFIC = {}   # {config_id: (bytes_per_launch, kernel_source_hash)}
+KERNEL_SOURCES = ["prefill_sigmoid_top_b200/csrc/gemm_bf16.cu", "prefill_sigmoid_top_b200/csrc/common.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--config", type=int, default=1)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--experts", type=int, default=0,
+                   help="override E (a smaller copy of the workload, e.g. for profiler captures)")
+    return p.parse_args(argv)
+
+
+def workload(args):
+    from prefill_sigmoid_top_b200 import inputs
+    cfg = inputs.CONFIGS[args.config]
+    if args.experts:
+        cfg = cfg.with_(E=args.experts, name=f"{cfg.name}_E{args.experts}")
+    return cfg
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (identity at world size 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, max_seconds: float, world: int) -> float:
+    """Whole-job throughput: units processed by all ranks / slowest rank's time."""
+    return per_rank_units * world / max_seconds
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload accounting
+def algorithmic_bytes(cfg, touched: int):
+    """Bytes the layer must move at minimum: touched experts' weights, router weights, x in, out."""
+    per_expert = 3 * cfg.I * cfg.H * 2
+    return dict(layer=touched * per_expert + cfg.E * cfg.H * 2 + 2 * cfg.M * cfg.H * 2,
+                up=touched * 2 * cfg.I * cfg.H * 2 + cfg.M * cfg.H * 2,
+                down=touched * cfg.I * cfg.H * 2,
+                finalize=cfg.M * cfg.K * cfg.H * 2 + 2 * cfg.M * cfg.H * 2)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import prefill_sigmoid_top_b200 as moe
+    from prefill_sigmoid_top_b200 import inputs
+
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    moe.library()  # fail loudly if the CUDA library cannot be loaded
+
+    cfg = workload(args)
+    if cfg.wdtype != "bf16":
+        raise SystemExit("the NVFP4 workload is not benchmarked by this build")
+    d = inputs.make_inputs(cfg, dev)
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    stream = torch.cuda.current_stream()
+
+    # buffers of the staged pass (the same kernels moe_layer launches)
+    route_ws = torch.empty(moe.route_workspace_size(shape), dtype=torch.uint8, device=dev)
+    ids = torch.empty(cfg.M, cfg.K, dtype=torch.int32, device=dev)
+    tw = torch.empty(cfg.M, cfg.K, dtype=torch.float32, device=dev)
+    cap = moe.align_capacity(shape)
+    plan = dict(sorted_ids=torch.empty(cap, dtype=torch.int32, device=dev),
+                block_expert=torch.empty(cap // cfg.B + 1, dtype=torch.int32, device=dev),
+                expert_counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+                expert_offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
+                num_tokens_post_padded=torch.empty(1, dtype=torch.int32, device=dev))
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    h = torch.empty(cap, cfg.I, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(cfg.M * cfg.K, cfg.H, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16, device=dev)
+
+    stages = ["route", "align", "up", "down", "finalize"]
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        moe.route(d["x"], d["w_router"], d["bias"], cfg.K, topk_ids=ids, topk_w=tw, ws=route_ws)
+        mark(1)
+        moe.align_block_size(ids, cfg.E, cfg.B, err_flag=err, out=plan)
+        mark(2)
+        moe.grouped_up_swiglu(d["x"], d["w_gate"], d["w_up"], plan, shape, h=h, err_flag=err)
+        mark(3)
+        moe.grouped_down(h, d["w_down"], plan, shape, y=y, err_flag=err)
+        mark(4)
+        moe.finalize_rmsnorm(d["x"], y, tw, d["gamma"], cfg.eps, out=out)
+        mark(5)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if moe.get_device_error(err) != 0:
+        raise SystemExit("device error during warm-up")
+    touched = int((plan["expert_counts"] > 0).sum().item())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t_wall0 = time.perf_counter()
+        for k in range(args.steps):
+            step(evs[k])
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall0
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = evs[0][0].elapsed_time(evs[-1][5])
+    stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, s in enumerate(stages)}
+    ms_per_step = total_ms / args.steps
+    max_s = reduce_max(total_ms / 1e3, world, dev)
+    value = aggregate(cfg.M * args.steps, max_s, world)
+
+    # ---- end to end through the public entry point (moe_layer) with host buffers
+    x_host = d["x"].cpu().pin_memory()
+    out_host = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    ws = torch.empty(moe.layer_workspace_size(shape), dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.layer(x_dev, d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"], cfg.eps, cfg.K,
+                  cfg.B, ws=ws, out=out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = reduce_max(e0.elapsed_time(e1) / 1e3, world, dev)
+    e2e_value = aggregate(cfg.M * args.steps, e2e_s, world)
+    # the e2e output equals the staged pass output
+    same = bool(torch.equal(out_host, out.cpu()))
+
+    hbm_peak, tc_peak, peak_kind = peaks()
+    ab = algorithmic_bytes(cfg, touched)
+    up_s = stage_ms["up"] / 1e3
+    achieved = ab["up"] / up_s / 1e9
+    traffic = None
+    tr = NCU_TRAFFIC.get(args.config)
+    if tr is not None and tr[1] == kernel_hash():
+        traffic = tr[0]
+    flops = 2.0 * 3 * cfg.H * cfg.I * cfg.M * cfg.K
+
+    result = {
+        "metric": "MoE layer tokens/s (decode/batch/prefill routed-MoE layer, H=7168 I=2048 E=256 top_k=16)",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_per_step,
+        "us_per_layer": ms_per_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights of the workload's shapes)",
+        "config": {"workload": cfg.name, "M": cfg.M, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.K,
+                   "block_size": cfg.B, "seed": cfg.seed, "router_bias": cfg.bias, "touched_experts": touched,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "no flush: each step streams GBs of expert weights, far above the 126 MB L2"},
+        "kernels_us": {s: v * 1e3 for s, v in stage_ms.items()},
+        "gpu_launches": 6 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "grouped_up_swiglu", "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
+                     "algorithmic_bytes": ab["up"], "peak_source": peak_kind},
+        "layer_roofline": {"algorithmic_bytes": ab["layer"], "GBps": ab["layer"] / (ms_per_step / 1e3) / 1e9,
+                           "frac_hbm": ab["layer"] / (ms_per_step / 1e3) / 1e9 / hbm_peak,
+                           "tflops": flops / (ms_per_step / 1e3) / 1e12,
+                           "frac_bf16_tensor": flops / (ms_per_step / 1e3) / 1e12 / tc_peak},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": cfg.M * cfg.H * 2,
+                "d2h_bytes_per_step": cfg.M * cfg.H * 2, "entry_point": "moe_layer", "matches_staged": same},
+        "wall_s_timed": t_wall,
+    }
+    cs = clocks.summary()
+    if cs is not None:
+        result["clocks"] = cs
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, d, target_s=12.0)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------------ oracle timing
+def _oracle_host_inputs(cfg, d):
+    import numpy as np
+    import oracle
+    from prefill_sigmoid_top_b200.inputs import bf16_bits
+    x, wr, b, g = bf16_bits(d["x"]), bf16_bits(d["w_router"]), d["bias"].cpu().numpy(), bf16_bits(d["gamma"])
+    ids, _ = oracle.route(x, wr, b, cfg.K)
+    need = sorted(set(int(e) for e in ids.ravel()))
+    wg, wu, wd = [None] * cfg.E, [None] * cfg.E, [None] * cfg.E
+    for e in need:
+        wg[e], wu[e], wd[e] = bf16_bits(d["w_gate"][e]), bf16_bits(d["w_up"][e]), bf16_bits(d["w_down"][e])
+    return x, wr, b, g, wg, wu, wd
+
+
+def cpu_baseline(cfg, d, target_s=12.0, max_tokens=None):
+    """Times the CPU oracle (as it stands) on a bounded sample of the same workload."""
+    import numpy as np
+    import oracle
+    x, wr, b, g, wg, wu, wd = _oracle_host_inputs(cfg, d)
+    n = cfg.M if max_tokens is None else min(cfg.M, max_tokens)
+    tokens_done, t0 = 0, time.perf_counter()
+    reps = 0
+    while True:
+        oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=np.arange(n, dtype=np.int32))
+        tokens_done += n
+        reps += 1
+        if time.perf_counter() - t0 >= target_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": tokens_done / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} x full layer on {n} of {cfg.M} tokens of {cfg.name} (fp64 C++ oracle, OpenMP), "
+                      f"{el:.1f} s"}
+
+
+def run_reference(args):
+    rank, local_rank, world = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle
+    cfg = workload(args)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    d = inputs.make_inputs(cfg, dev)
+    x, wr, b, g, wg, wu, wd = _oracle_host_inputs(cfg, d)
+    del d
+    # size one step so that the whole run stays within a few minutes
+    t0 = time.perf_counter()
+    oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=np.arange(1, dtype=np.int32))
+    per_token = time.perf_counter() - t0
+    budget_per_step = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(cfg.M, budget_per_step // max(per_token, 1e-3))))
+    toks = np.arange(n, dtype=np.int32)
+    for _ in range(args.warmup):
+        oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=toks)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=toks)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    sample = f"{n} of {cfg.M} tokens of {cfg.name} per step (fp64 C++ oracle, OpenMP)"
+    print(json.dumps({
+        "impl": "reference", "metric": "MoE layer tokens/s (decode/batch/prefill routed-MoE layer, H=7168 I=2048 "
+                                      "E=256 top_k=16)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": cfg.name, "M": cfg.M, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.K,
+                   "block_size": cfg.B, "seed": cfg.seed},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
