@@ -20,7 +20,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -30,9 +29,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 # ncu DRAM traffic of the dominant kernel, per launch, measured on the decode
-# workload (profiles/grouped_up_decode_m8.md).  Valid only while the kernel
+# workload (profiles/grouped_up_decode_m8_E32.md).  Valid only while the kernel
 # sources hash to KERNEL_HASH; otherwise "traffic" is reported as null.
-NCU_TRAFFIC = {}   # {config_id: (bytes_per_launch, kernel_source_hash)}
+NCU_TRAFFIC = {
+    # decode M=8: E=32 capture (1.8246 GB for 31 touched experts) scaled to 95 touched experts
+    1: (5_591_000_000, "9d3b0736d6de6a3e"),
+}
 KERNEL_SOURCES = ["prefill_sigmoid_top_b200/csrc/gemm_bf16.cu", "prefill_sigmoid_top_b200/csrc/common.cuh"]
 
 
@@ -88,59 +90,63 @@ def aggregate(per_rank_units: float, max_seconds: float, world: int) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML
+    every 2 ms while the timed region runs (read-only queries)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device_index: int, period_s: float = 0.002):
+        self.dev = torch_device_index
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop.is_set():
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(get_reasons(h))))
+                time.sleep(self.period)
+            nv.nvmlShutdown()
+        except Exception as e:  # no NVML: report no clock record rather than fail the bench
+            self.error = repr(e)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
-            self._t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        time.sleep(0.01)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        self._thread.join(timeout=5)
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ workload accounting
@@ -278,7 +284,7 @@ def run_ours(args):
     up_s = stage_ms["up"] / 1e3
     achieved = ab["up"] / up_s / 1e9
     traffic = None
-    tr = NCU_TRAFFIC.get(args.config)
+    tr = NCU_TRAFFIC.get(args.config) if not args.experts else None
     if tr is not None and tr[1] == kernel_hash():
         traffic = tr[0]
     flops = 2.0 * 3 * cfg.H * cfg.I * cfg.M * cfg.K

@@ -57,16 +57,16 @@ def lib():
                 "oracle_topk": (None, [vp, i32, i32, i32, vp, vp]),
                 "oracle_align": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
                 "oracle_expert": (None, [vp, vp, vp, vp, i32, i32, vp, vp]),
-                "oracle_finalize": (None, [vp, vp, vp, vp, f64, i32, i32, i32, vp, vp]),
+                "oracle_finalize": (None, [vp, vp, vp, vp, f64, i32, i32, i32, vp, vp, vp, vp]),
                 "oracle_layer": (i32, [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, vp, i32,
-                                       vp, vp, vp, vp, vp, vp]),
+                                       vp, vp, vp, vp, vp, vp, vp, vp]),
                 "oracle_dense_mixture": (None, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]),
                 "oracle_nvfp4_global_scale": (f32, [f32]),
                 "oracle_nvfp4_quantize": (None, [vp, i64, i64, f32, vp, vp]),
                 "oracle_nvfp4_quantize_bf16": (f32, [vp, i64, i64, vp, vp]),
                 "oracle_nvfp4_dequantize": (None, [vp, vp, i64, i64, f32, vp]),
                 "oracle_layer_nvfp4": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32,
-                                             i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp]),
+                                             i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
                 "oracle_num_threads": (i32, []),
             }
             for name, (res, args) in sig.items():
@@ -182,15 +182,18 @@ def expert(x_row, w_gate_e, w_up_e, w_down_e):
     return h, y
 
 
-def finalize(x, y, w, gamma, eps, want_residual=True):
-    """x [M,H] bf16 bits, y [M,K,H] bf16 bits, w [M,K] float -> (out, residual) bf16 bits."""
+def finalize(x, y, w, gamma, eps, want_residual=True, want_f64=False):
+    """x [M,H] bf16 bits, y [M,K,H] bf16 bits, w [M,K] float -> (out, residual) bf16 bits
+    (and, if asked, the same two before their final bf16 rounding, as float64)."""
     x, y, gamma = _u16(x), _u16(y), _u16(gamma)
     w = np.ascontiguousarray(w, dtype=np.float64)
     M, K, H = y.shape
     out = np.empty((M, H), np.uint16)
     res = np.empty((M, H), np.uint16) if want_residual else None
-    lib().oracle_finalize(_p(x), _p(y), _p(w), _p(gamma), float(eps), M, K, H, _p(out), _p(res))
-    return out, res
+    o64 = np.empty((M, H), np.float64) if want_f64 else None
+    s64 = np.empty((M, H), np.float64) if want_f64 else None
+    lib().oracle_finalize(_p(x), _p(y), _p(w), _p(gamma), float(eps), M, K, H, _p(out), _p(res), _p(o64), _p(s64))
+    return (out, res, o64, s64) if want_f64 else (out, res)
 
 
 def layer(x, w_router, bias, w_gate, w_up, w_down, gamma, eps, K, tokens=None, want_h=False):
@@ -216,11 +219,14 @@ def layer(x, w_router, bias, w_gate, w_up, w_down, gamma, eps, K, tokens=None, w
     y = np.empty((n, K, H), np.uint16)
     out = np.empty((n, H), np.uint16)
     res = np.empty((n, H), np.uint16)
+    o64 = np.empty((n, H), np.float64)
+    s64 = np.empty((n, H), np.float64)
     st = lib().oracle_layer(_p(x), _p(w_router), _p(b), _ptr_table(wg), _ptr_table(wu), _ptr_table(wd), _p(gamma),
-                            float(eps), M, H, I, E, K, _p(tok), n, _p(ids), _p(w), _p(h), _p(y), _p(out), _p(res))
+                            float(eps), M, H, I, E, K, _p(tok), n, _p(ids), _p(w), _p(h), _p(y), _p(out), _p(res),
+                            _p(o64), _p(s64))
     if st != 0:
         raise RuntimeError(f"oracle_layer status {st}")
-    return dict(ids=ids, w=w, h=h, y=y, out=out, residual=res, tokens=tok)
+    return dict(ids=ids, w=w, h=h, y=y, out=out, residual=res, out_f64=o64, residual_f64=s64, tokens=tok)
 
 
 def dense_mixture(x, w_gate, w_up, w_down, wdense):
@@ -297,9 +303,12 @@ def layer_nvfp4(x, w_router, bias, gate_q, up_q, down_q, gamma, eps, K, tokens=N
     y = np.empty((n, K, H), np.uint16)
     out = np.empty((n, H), np.uint16)
     res = np.empty((n, H), np.uint16)
+    o64 = np.empty((n, H), np.float64)
+    s64 = np.empty((n, H), np.float64)
     st = lib().oracle_layer_nvfp4(_p(x), _p(w_router), _p(b), gc, gsc, _p(ggs), uc, usc, _p(ugs), dc, dsc, _p(dgs),
                                   _p(gamma), float(eps), M, H, I, E, K, _p(tok), n, _p(ids), _p(w), _p(h), _p(y),
-                                  _p(out), _p(res))
+                                  _p(out), _p(res), _p(o64), _p(s64))
     if st != 0:
         raise RuntimeError(f"oracle_layer_nvfp4 status {st}")
-    return dict(ids_all=ids, w_all=w, h_all=h, y=y, out=out, residual=res, tokens=tok)
+    return dict(ids_all=ids, w_all=w, h_all=h, y=y, out=out, residual=res, out_f64=o64, residual_f64=s64,
+                tokens=tok)

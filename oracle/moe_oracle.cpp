@@ -329,8 +329,15 @@ void oracle_expert(const uint16_t* x, const uint16_t* w_gate, const uint16_t* w_
 //   s = x + sum_k w_k * y_k             (fp64)
 //   out = bf16( s / sqrt(mean_h(s^2) + eps) * gamma )
 //   residual_out = bf16(s)              (nullable)
+// out64 / s64 (nullable) receive the same two values before their final bf16
+// rounding: the reference for tolerance comparisons of the layer output
+// (reading: the bf16 quantisation the reference applies is that of the stored
+// intermediates h and y; the output's own rounding is part of the error
+// measured, since two correct bf16 roundings of values that straddle a
+// rounding boundary differ by a whole bf16 step).
 void oracle_finalize_token(const uint16_t* x, const uint16_t* y, const double* w, const uint16_t* gamma,
-                           double eps, int K, int H, uint16_t* out, uint16_t* residual_out) {
+                           double eps, int K, int H, uint16_t* out, uint16_t* residual_out, double* out64,
+                           double* s64) {
   std::vector<double> s(H);
   for (int c = 0; c < H; ++c) {
     double acc = bf16_value(x[c]);
@@ -341,20 +348,26 @@ void oracle_finalize_token(const uint16_t* x, const uint16_t* y, const double* w
   for (int c = 0; c < H; ++c) ss += s[c] * s[c];
   const double inv = 1.0 / std::sqrt(ss / H + eps);
   for (int c = 0; c < H; ++c) {
-    out[c] = bf16_round(s[c] * inv * bf16_value(gamma[c]));
+    const double o = s[c] * inv * bf16_value(gamma[c]);
+    out[c] = bf16_round(o);
     if (residual_out) residual_out[c] = bf16_round(s[c]);
+    if (out64) out64[c] = o;
+    if (s64) s64[c] = s[c];
   }
 }
 
 // Finalize over M tokens: y is [M,K,H] bf16, w is [M,K] fp64.
 void oracle_finalize(const uint16_t* x, const uint16_t* y, const double* w, const uint16_t* gamma,
-                     double eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out) {
+                     double eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out, double* out64,
+                     double* s64) {
 #pragma omp parallel for schedule(static)
   for (int t = 0; t < M; ++t)
     oracle_finalize_token(x + static_cast<size_t>(t) * H, y + static_cast<size_t>(t) * K * H,
                           w + static_cast<size_t>(t) * K, gamma, eps, K, H,
                           out + static_cast<size_t>(t) * H,
-                          residual_out ? residual_out + static_cast<size_t>(t) * H : nullptr);
+                          residual_out ? residual_out + static_cast<size_t>(t) * H : nullptr,
+                          out64 ? out64 + static_cast<size_t>(t) * H : nullptr,
+                          s64 ? s64 + static_cast<size_t>(t) * H : nullptr);
 }
 
 // The whole layer for a chosen subset of tokens.  Expert weights are passed
@@ -371,7 +384,7 @@ int oracle_layer(const uint16_t* x, const uint16_t* w_router, const float* bias,
                  const uint16_t* const* w_down, const uint16_t* gamma, float eps,
                  int M, int H, int I, int E, int K, const int32_t* tokens, int n_tokens,
                  int32_t* topk_ids, double* topk_w, uint16_t* h_out, uint16_t* y_out,
-                 uint16_t* out, uint16_t* residual_out) {
+                 uint16_t* out, uint16_t* residual_out, double* out64, double* s64) {
   (void)M;
   std::vector<float> z(static_cast<size_t>(E));
   for (int i = 0; i < n_tokens; ++i) {
@@ -403,7 +416,9 @@ int oracle_layer(const uint16_t* x, const uint16_t* w_router, const float* bias,
       oracle_finalize_token(x + static_cast<size_t>(tokens[i]) * H, y + static_cast<size_t>(i) * K * H,
                             topk_w + static_cast<size_t>(i) * K, gamma, static_cast<double>(eps), K, H,
                             out + static_cast<size_t>(i) * H,
-                            residual_out ? residual_out + static_cast<size_t>(i) * H : nullptr);
+                            residual_out ? residual_out + static_cast<size_t>(i) * H : nullptr,
+                            out64 ? out64 + static_cast<size_t>(i) * H : nullptr,
+                            s64 ? s64 + static_cast<size_t>(i) * H : nullptr);
   }
   return 0;
 }
@@ -500,7 +515,8 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
                        const uint8_t* const* down_codes, const uint8_t* const* down_scales, const float* down_gs,
                        const uint16_t* gamma, float eps, int M, int H, int I, int E, int K,
                        const int32_t* tokens, int n_tokens, int32_t* topk_ids_all, double* topk_w_all,
-                       uint16_t* h_all, uint16_t* y_out, uint16_t* out, uint16_t* residual_out) {
+                       uint16_t* h_all, uint16_t* y_out, uint16_t* out, uint16_t* residual_out,
+                       double* out64, double* s64) {
   // routing for every token (h needs all of them)
   std::vector<float> z(static_cast<size_t>(M) * E);
   oracle_router_logits(x, w_router, bias, M, H, E, z.data(), nullptr);
@@ -574,7 +590,9 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
       oracle_finalize_token(x + static_cast<size_t>(tokens[i]) * H, y + static_cast<size_t>(i) * K * H,
                             topk_w_all + static_cast<size_t>(tokens[i]) * K, gamma, static_cast<double>(eps), K, H,
                             out + static_cast<size_t>(i) * H,
-                            residual_out ? residual_out + static_cast<size_t>(i) * H : nullptr);
+                            residual_out ? residual_out + static_cast<size_t>(i) * H : nullptr,
+                            out64 ? out64 + static_cast<size_t>(i) * H : nullptr,
+                            s64 ? s64 + static_cast<size_t>(i) * H : nullptr);
   }
   return 0;
 }
