@@ -56,6 +56,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--experts", type=int, default=0,
                    help="override E (a smaller copy of the workload, e.g. for profiler captures)")
+    p.add_argument("--tokens", type=int, default=0, help="override M (with --experts: a smaller copy)")
+    p.add_argument("--topk", type=int, default=0, help="override top_k (with --experts)")
     return p.parse_args(argv)
 
 
@@ -64,6 +66,10 @@ def workload(args):
     cfg = inputs.CONFIGS[args.config]
     if args.experts:
         cfg = cfg.with_(E=args.experts, name=f"{cfg.name}_E{args.experts}")
+    if args.tokens:
+        cfg = cfg.with_(M=args.tokens, name=f"{cfg.name}_M{args.tokens}")
+    if args.topk:
+        cfg = cfg.with_(K=args.topk, name=f"{cfg.name}_K{args.topk}")
     return cfg
 
 
@@ -204,6 +210,8 @@ def run_ours(args):
                 expert_offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
                 num_tokens_post_padded=torch.empty(1, dtype=torch.int32, device=dev))
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    up_ws_bytes = moe.up_workspace_size(shape)
+    up_ws = torch.empty(up_ws_bytes, dtype=torch.uint8, device=dev) if up_ws_bytes else None
     h = torch.empty(cap, cfg.I, dtype=torch.bfloat16, device=dev)
     y = torch.empty(cfg.M * cfg.K, cfg.H, dtype=torch.bfloat16, device=dev)
     out = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16, device=dev)
@@ -219,7 +227,7 @@ def run_ours(args):
         mark(1)
         moe.align_block_size(ids, cfg.E, cfg.B, err_flag=err, out=plan)
         mark(2)
-        moe.grouped_up_swiglu(d["x"], d["w_gate"], d["w_up"], plan, shape, h=h, err_flag=err)
+        moe.grouped_up_swiglu(d["x"], d["w_gate"], d["w_up"], plan, shape, h=h, err_flag=err, ws=up_ws)
         mark(3)
         moe.grouped_down(h, d["w_down"], plan, shape, y=y, err_flag=err)
         mark(4)
@@ -284,7 +292,7 @@ def run_ours(args):
     up_s = stage_ms["up"] / 1e3
     achieved = ab["up"] / up_s / 1e9
     traffic = None
-    tr = NCU_TRAFFIC.get(args.config) if not args.experts else None
+    tr = NCU_TRAFFIC.get(args.config) if not (args.experts or args.tokens or args.topk) else None
     if tr is not None and tr[1] == kernel_hash():
         traffic = tr[0]
     flops = 2.0 * 3 * cfg.H * cfg.I * cfg.M * cfg.K

@@ -140,8 +140,10 @@ MOE_API size_t moe_align_capacity(moe_shape_t s); /* M*top_k + E*(block_size-1) 
  *   g = x[t] . w.gate[e]^T,  u = x[t] . w.up[e]^T   (fp32 accumulation)
  *   h[r, :] = bf16(silu(g) * u),   silu(g) = g / (1 + exp(-g))
  * h: bf16 [moe_align_capacity(s), I]; padding rows are not written.
- * MOE_W_NVFP4 quantises x on the fly into ws (moe_up_workspace_size bytes);
- * for MOE_W_BF16 ws may be NULL. */
+ * ws (nullable): moe_up_workspace_size(s, dtype) bytes of device scratch.  With
+ * it, wide token tiles first gather x into plan order there and read it as
+ * contiguous rows; without it the rows are gathered inside the GEMM.  Both
+ * give the same result.  MOE_W_NVFP4 quantises x on the fly into ws. */
 MOE_API moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
                                    moe_shape_t s, moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err_flag,
                                    moe_stream_t stream);

@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "MoEError", "Shape", "library", "route", "align_block_size", "grouped_up_swiglu", "grouped_down",
-    "finalize_rmsnorm", "layer", "layer_workspace_size", "layer_workspace_layout", "align_capacity",
+    "finalize_rmsnorm", "layer", "layer_workspace_size", "up_workspace_size", "layer_workspace_layout", "align_capacity",
     "route_workspace_size", "get_device_error", "status_string", "STATUS",
 ]
 
@@ -219,15 +219,23 @@ def _plan_struct(plan):
                  plan["expert_offsets"].data_ptr(), plan["num_tokens_post_padded"].data_ptr())
 
 
-def grouped_up_swiglu(x, w_gate, w_up, plan, shape: Shape, h=None, err_flag=None):
+def up_workspace_size(shape: Shape, wdtype: int = MOE_W_BF16) -> int:
+    return int(library().moe_up_workspace_size(shape.c(), wdtype))
+
+
+def grouped_up_swiglu(x, w_gate, w_up, plan, shape: Shape, h=None, err_flag=None, ws=None):
     """h[cap, I] = bf16(silu(x W_gate^T) * (x W_up^T)) in plan order."""
     _need_cuda(x, w_gate, w_up)
     if h is None:
         h = torch.empty(align_capacity(shape), shape.I, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        need = up_workspace_size(shape)
+        ws = torch.empty(need, dtype=torch.uint8, device=x.device) if need else None
     w = _weights_struct(w_gate, w_up, w_up)
     p = _plan_struct(plan)
     _check(library().moe_grouped_up_swiglu(_ptr(_bf16(x)), ctypes.byref(w), ctypes.byref(p), shape.c(), _ptr(h),
-                                           None, 0, _ptr(err_flag), _stream()), "moe_grouped_up_swiglu")
+                                           _ptr(ws), 0 if ws is None else ws.numel(), _ptr(err_flag), _stream()),
+           "moe_grouped_up_swiglu")
     return h
 
 

@@ -67,13 +67,16 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
-// Token-tile width of the grouped kernels: the mean routed rows per expert
-// decides between the decode shape (32) and the batch/prefill shape (128).
-// MOE_GEMM_NMAX=32|128 overrides (used by tests to cover both shapes).
+// Token-tile width of the grouped kernels, from the mean routed rows per
+// expert (known on the host without reading the plan back): decode shapes
+// (<= 24) use 32-row tiles, larger ones 128-row tiles.  256-row tiles measured
+// slower on the batch and prefill workloads (one accumulator set fills tensor
+// memory), so they run only when asked for.  MOE_GEMM_NMAX=32|128|256
+// overrides (the tests cover every variant).
 int choose_nmax(const moe_shape_t& s) {
   if (const char* env = std::getenv("MOE_GEMM_NMAX")) {
     const int v = std::atoi(env);
-    if (v == 32 || v == 128) return v;
+    if (v == 32 || v == 128 || v == 256) return v;
   }
   const double per_expert = static_cast<double>(s.M) * s.top_k / s.E;
   return per_expert <= 24.0 ? 32 : 128;
@@ -81,6 +84,51 @@ int choose_nmax(const moe_shape_t& s) {
 
 size_t cap_rows(const moe_shape_t& s) {
   return static_cast<size_t>(s.M) * s.top_k + static_cast<size_t>(s.E) * (s.block_size - 1);
+}
+
+// Whether the up projection first gathers x into plan order (one pass over
+// the routed rows) and then reads it as contiguous 16-row boxes, instead of
+// gathering the rows inside the GEMM with tile::gather4.  The in-GEMM gather
+// issues one copy per 4 rows per 64-column stage, which limits the wide
+// token tiles; the decode tiles (<= 32 rows) keep it.  MOE_UP_GATHER=tma |
+// pregather overrides.
+bool want_pregather(const moe_shape_t& s) {
+  if (const char* env = std::getenv("MOE_UP_GATHER")) {
+    if (std::strcmp(env, "tma") == 0) return false;
+    if (std::strcmp(env, "pregather") == 0) return true;
+  }
+  return choose_nmax(s) >= 128;
+}
+
+size_t pregather_bytes(const moe_shape_t& s) { return align_up(cap_rows(s) * s.H * sizeof(uint16_t)); }
+
+// Whether the batch/prefill shapes run the persistent kernel (one CTA per SM,
+// deep weight ring, double-buffered accumulators).  MOE_GEMM_PERSISTENT=0|1
+// overrides; the up projection also needs the plan-ordered copy of x, so it
+// only takes this path when the caller provides that workspace.
+bool want_persistent(const moe_shape_t& s) {
+  if (const char* env = std::getenv("MOE_GEMM_PERSISTENT")) {
+    if (std::strcmp(env, "0") == 0) return false;
+    if (std::strcmp(env, "1") == 0) return true;
+  }
+  return choose_nmax(s) >= 128;
+}
+
+// Ring shape of the persistent kernels (MOE_PGEMM_DEEP_B=1: 4 weight + 5
+// token-row stages; default 5 + 3).
+bool deep_token_ring() {
+  const char* env = std::getenv("MOE_PGEMM_DEEP_B");
+  return env != nullptr && std::strcmp(env, "1") == 0;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cached[64] = {};
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
 }
 
 moe_status_t check_plan(const moe_plan_t* p) {
@@ -97,12 +145,24 @@ moe_status_t check_bf16_weights(const moe_weights_t* w) {
 }
 
 moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
-                    moe_bf16_t* h, int32_t* err, cudaStream_t stream) {
+                    moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t stream) {
   CUtensorMap mg, mu, mx;
   const uint64_t rows = static_cast<uint64_t>(s.E) * s.I;
-  if (!make_map_bf16(&mg, w->gate, rows, s.H, 128) || !make_map_bf16(&mu, w->up, rows, s.H, 128) ||
-      !make_map_bf16(&mx, x, s.M, s.H, 1))
+  const bool have_ws = ws != nullptr && ws_bytes >= pregather_bytes(s) && aligned16(ws) &&
+                       plan->num_tokens_post_padded != nullptr;
+  const bool persistent = want_persistent(s);
+  const bool gathered = want_pregather(s) && have_ws;
+  if (!make_map_bf16(&mg, w->gate, rows, s.H, 128) || !make_map_bf16(&mu, w->up, rows, s.H, 128))
     return MOE_ERR_CUDA;
+  if (gathered) {
+    auto* xg = static_cast<moe_bf16_t*>(ws);
+    const cudaError_t e = moe::launch_gather_rows(x, plan->sorted_ids, plan->num_tokens_post_padded, s.M, s.top_k,
+                                                  s.H, static_cast<int>(cap_rows(s)), xg, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (!make_map_bf16(&mx, xg, cap_rows(s), s.H, persistent ? 32 : 16)) return MOE_ERR_CUDA;
+  } else if (!make_map_bf16(&mx, x, s.M, s.H, 1)) {
+    return MOE_ERR_CUDA;
+  }
   GroupedGemmArgs a{};
   a.sorted_ids = plan->sorted_ids;
   a.expert_counts = plan->expert_counts;
@@ -115,14 +175,18 @@ moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_
   a.rows_per_expert = s.I;
   a.kdim = s.H;
   a.out_ld = s.I;
-  return cuda_status(moe::launch_grouped_up(mg, mu, mx, a, choose_nmax(s), stream));
+  if (persistent)
+    return cuda_status(
+        moe::launch_persistent_up(mg, mu, mx, a, choose_nmax(s), !gathered, deep_token_ring(), num_sms(), stream));
+  return cuda_status(moe::launch_grouped_up(mg, mu, mx, a, choose_nmax(s), gathered, stream));
 }
 
 moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
                       moe_bf16_t* y, int32_t* err, cudaStream_t stream) {
   CUtensorMap md, mh;
+  const bool persistent = want_persistent(s);
   if (!make_map_bf16(&md, w->down, static_cast<uint64_t>(s.E) * s.H, s.I, 128) ||
-      !make_map_bf16(&mh, h, cap_rows(s), s.I, 16))
+      !make_map_bf16(&mh, h, cap_rows(s), s.I, persistent ? 32 : 16))
     return MOE_ERR_CUDA;
   GroupedGemmArgs a{};
   a.sorted_ids = plan->sorted_ids;
@@ -136,6 +200,8 @@ moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_pla
   a.rows_per_expert = s.H;
   a.kdim = s.I;
   a.out_ld = s.H;
+  if (persistent)
+    return cuda_status(moe::launch_persistent_down(md, mh, a, choose_nmax(s), deep_token_ring(), num_sms(), stream));
   return cuda_status(moe::launch_grouped_down(md, mh, a, choose_nmax(s), stream));
 }
 
@@ -167,7 +233,8 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   off = align_up(off + cap * s.I * sizeof(uint16_t));
   L.y = off;
   off = align_up(off + mk * s.H * sizeof(uint16_t));
-  L.act_scratch = off;
+  L.act_scratch = off;  // x gathered into plan order (up projection)
+  off = align_up(off + pregather_bytes(s));
   L.total = off;
   return L;
 }
@@ -201,7 +268,8 @@ size_t moe_route_workspace_size(moe_shape_t s) {
 
 size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK) return 0;
-  return dtype == MOE_W_BF16 ? 0 : 0;
+  (void)dtype;
+  return (want_pregather(s) || want_persistent(s)) ? pregather_bytes(s) : 0;
 }
 
 size_t moe_down_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
@@ -238,15 +306,13 @@ moe_status_t moe_align_block_size(const int32_t* topk_ids, moe_shape_t s, int32_
 moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
                                    moe_shape_t s, moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err_flag,
                                    moe_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   moe_status_t st = check_shape(s);
   if (st != MOE_OK) return st;
   if ((st = check_bf16_weights(w)) != MOE_OK) return st;
   if ((st = check_plan(plan)) != MOE_OK) return st;
   if (!x || !h || !w->gate || !w->up) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(h) || !aligned16(w->gate) || !aligned16(w->up)) return MOE_ERR_INVALID_ARG;
-  return run_up(x, w, plan, s, h, err_flag, static_cast<cudaStream_t>(stream));
+  return run_up(x, w, plan, s, h, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_grouped_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, moe_shape_t s,
@@ -325,7 +391,7 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
                                           err, cs))) != MOE_OK)
     return st;
   moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
-  if ((st = run_up(x, w, &plan, s, h, err, cs)) != MOE_OK) return st;
+  if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
   if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
   return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
 }

@@ -55,14 +55,20 @@ struct Cfg {
   static constexpr int kAPerStage = kUp ? 2 : 1;
   static constexpr int kStageBytes = kATile * kAPerStage + kBTile;
   static constexpr int kTmemCols = pow2_at_least(kUp ? 2 * kNmax : kNmax);
-  static constexpr int kMiscBytes = 1024;
+  static constexpr int kMiscBytes = (128 + 4 * kNmax + 1023) / 1024 * 1024;  // barriers, flags, token ids
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMiscBytes;
   static_assert(kBTile % 1024 == 0, "token tile must keep 1024-byte alignment");
   static_assert(kNmax % 16 == 0 && kNmax <= 256, "MMA N limits");
-  static_assert(kTmemCols <= 256, "two CTAs per SM share the 512 tensor-memory columns");
+  static_assert(kTmemCols <= 512, "tensor memory has 512 columns");
+  // A CTA that takes more than half of tensor memory must also take more than
+  // half of shared memory, so that no second CTA is resident to wait on it.
+  static_assert(kTmemCols <= 256 || kSmemBytes > 116 * 1024, "tensor memory / occupancy mismatch");
 };
 
-template <bool kUp, int kNmax, int kStages>
+// kGatherB: the token rows of the B operand are gathered from x by token id
+// (tile::gather4); otherwise they are consecutive plan rows of a tensor that
+// is already in plan order (h, or x gathered by gather_rows_kernel).
+template <bool kUp, int kNmax, int kStages, bool kGatherB>
 __global__ void __launch_bounds__(128, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                         const __grid_constant__ CUtensorMap tm_b, const GroupedGemmArgs args) {
@@ -76,28 +82,32 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* accf = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* info = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 1));  // [0] expert, [1] local tile
-  int* tok = info + 2;                                                           // [kNmax]
+  int* info = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 1));  // expert, token tile, weight tile
+  int* tok = info + 4;                                                           // [kNmax]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wt = blockIdx.x;
-  const int tile = blockIdx.y;
   const int E = args.E;
+  const int W = args.rows_per_expert / kBM;  // weight tiles per expert
 
-  // ---- which expert / which of its tiles is token tile `tile`
+  // ---- which (expert, weight tile, token tile) this CTA computes.  CTAs are
+  // ordered expert by expert, then weight tile, then token tile (fastest), so
+  // the token tiles that stream the same weight panel start together and the
+  // panel is fetched from HBM once and shared through L2.
   int* cnt = reinterpret_cast<int*>(stages);  // scratch before the pipeline starts (E <= 1024)
   for (int e = tid; e < E; e += 128) cnt[e] = args.expert_counts[e];
   if (tid == 0) {
     info[0] = -1;
     info[1] = 0;
+    info[2] = 0;
     *abort_flag = 0;
   }
   __syncthreads();
   if (warp == 0) {
+    const int linear = blockIdx.x;
     const int per = (E + 31) / 32;
     const int lo = min(E, lane * per), hi = min(E, lo + per);
     int sum = 0;
-    for (int e = lo; e < hi; ++e) sum += (cnt[e] + kNmax - 1) / kNmax;
+    for (int e = lo; e < hi; ++e) sum += W * ((cnt[e] + kNmax - 1) / kNmax);
     int incl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -105,16 +115,18 @@ __global__ void __launch_bounds__(128, 1)
       if (lane >= off) incl += v;
     }
     const int excl = incl - sum;
-    if (tile >= excl && tile < incl) {
+    if (linear >= excl && linear < incl) {
       int t = excl;
       for (int e = lo; e < hi; ++e) {
-        const int n = (cnt[e] + kNmax - 1) / kNmax;
-        if (tile < t + n) {
+        const int ntiles = (cnt[e] + kNmax - 1) / kNmax;
+        if (linear < t + W * ntiles) {
+          const int rel = linear - t;
           info[0] = e;
-          info[1] = tile - t;
+          info[1] = rel % ntiles;
+          info[2] = rel / ntiles;
           break;
         }
-        t += n;
+        t += W * ntiles;
       }
     }
   }
@@ -122,16 +134,18 @@ __global__ void __launch_bounds__(128, 1)
   const int e = info[0];
   if (e < 0) return;  // past the real tile count: the whole CTA leaves before any async work
   const int local = info[1];
-  const int nrows = min(kNmax, cnt[e] - local * kNmax);
+  const int wt = info[2];
+  const int count_e = cnt[e];
+  const int nrows = min(kNmax, count_e - local * kNmax);
   const int row0 = args.expert_offsets[e] + local * kNmax;
   const int N = (nrows + 15) & ~15;
   const int nslots = args.M * args.top_k;
   for (int n = tid; n < N; n += 128) {
-    int v = kUp ? 0 : -1;
+    int v = (kUp && kGatherB) ? 0 : -1;
     if (n < nrows) {
       const int id = args.sorted_ids[row0 + n];
       if (id >= 0 && id < nslots) {
-        v = kUp ? id / args.top_k : id;
+        v = (kUp && kGatherB) ? id / args.top_k : id;
       } else {
         set_error(args.err, kErrInvalidInput);
       }
@@ -166,7 +180,11 @@ __global__ void __launch_bounds__(128, 1)
       if (kUp) prefetch_tensor_map(&tm_a1);
       prefetch_tensor_map(&tm_b);
     }
-    const uint64_t pol_w = l2_policy_evict_first();
+    // A weight panel used by one token tile only is streamed with an
+    // evict-first hint; an expert with several token tiles re-reads its panel
+    // from L2, so those loads keep the normal policy.
+    const bool single_use = count_e <= kNmax;
+    const uint64_t pol_w = single_use ? l2_policy_evict_first() : l2_policy_evict_normal();
     int issued = 0;
     for (int k = 0; k < nk; ++k) {
       const int s = k % kStages;
@@ -189,7 +207,7 @@ __global__ void __launch_bounds__(128, 1)
         if (kUp) tma_load_2d_hint(&tm_a1, &full[s], st + kATile, k * kBK, a_row, pol_w);
       }
       __syncwarp();
-      if (kUp) {
+      if (kGatherB) {
         for (int i = lane; i < N / 4; i += 32)
           tma_gather4(&tm_b, &full[s], bt + i * 4 * (kBK * 2), k * kBK, tok[4 * i], tok[4 * i + 1], tok[4 * i + 2],
                       tok[4 * i + 3]);
@@ -290,11 +308,11 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <bool kUp, int kNmax, int kStages>
+template <bool kUp, int kNmax, int kStages, bool kGatherB>
 cudaError_t launch_variant(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                            const GroupedGemmArgs& args, cudaStream_t stream) {
   using C = Cfg<kUp, kNmax, kStages>;
-  auto kern = grouped_gemm_kernel<kUp, kNmax, kStages>;
+  auto kern = grouped_gemm_kernel<kUp, kNmax, kStages, kGatherB>;
   int dev = 0;
   cudaError_t st = cudaGetDevice(&dev);
   if (st != cudaSuccess) return st;
@@ -306,23 +324,52 @@ cudaError_t launch_variant(const CUtensorMap& a0, const CUtensorMap& a1, const C
   }
   const long long mk = static_cast<long long>(args.M) * args.top_k;
   const long long tiles_ub = mk / kNmax + (mk < args.E ? mk : args.E);
-  dim3 grid(args.rows_per_expert / kBM, static_cast<unsigned>(tiles_ub));
+  const unsigned grid = static_cast<unsigned>((args.rows_per_expert / kBM) * tiles_ub);
   kern<<<grid, 128, C::kSmemBytes, stream>>>(a0, a1, b, args);
   return cudaGetLastError();
+}
+
+// xg[r, :] = x[sorted_ids[r] / top_k, :] for every real plan row r (padding
+// rows are skipped): one warp per row, 16-byte loads and stores.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, const int32_t* sorted_ids,
+                                                          const int32_t* ntpp, int nslots, int top_k, int row_vecs,
+                                                          int cap, uint4* __restrict__ xg) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= cap || r >= *ntpp) return;
+  const int id = sorted_ids[r];
+  if (id < 0 || id >= nslots) return;
+  const uint4* src = x + static_cast<size_t>(id / top_k) * row_vecs;
+  uint4* dst = xg + static_cast<size_t>(r) * row_vecs;
+  for (int i = lane; i < row_vecs; i += 32) dst[i] = src[i];
 }
 
 }  // namespace
 
 cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
-                              const GroupedGemmArgs& args, int nmax, cudaStream_t stream) {
-  if (nmax <= 32) return launch_variant<true, 32, 3>(w_gate, w_up, x_rows, args, stream);
-  return launch_variant<true, 128, 2>(w_gate, w_up, x_rows, args, stream);
+                              const GroupedGemmArgs& args, int nmax, bool gathered, cudaStream_t stream) {
+  if (gathered) {
+    if (nmax <= 32) return launch_variant<true, 32, 3, false>(w_gate, w_up, x_rows, args, stream);
+    if (nmax <= 128) return launch_variant<true, 128, 2, false>(w_gate, w_up, x_rows, args, stream);
+    return launch_variant<true, 256, 3, false>(w_gate, w_up, x_rows, args, stream);
+  }
+  if (nmax <= 32) return launch_variant<true, 32, 3, true>(w_gate, w_up, x_rows, args, stream);
+  if (nmax <= 128) return launch_variant<true, 128, 2, true>(w_gate, w_up, x_rows, args, stream);
+  return launch_variant<true, 256, 3, true>(w_gate, w_up, x_rows, args, stream);
 }
 
 cudaError_t launch_grouped_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
                                 int nmax, cudaStream_t stream) {
-  if (nmax <= 32) return launch_variant<false, 32, 5>(w_down, w_down, h_rows, args, stream);
-  return launch_variant<false, 128, 3>(w_down, w_down, h_rows, args, stream);
+  if (nmax <= 32) return launch_variant<false, 32, 5, false>(w_down, w_down, h_rows, args, stream);
+  if (nmax <= 128) return launch_variant<false, 128, 3, false>(w_down, w_down, h_rows, args, stream);
+  return launch_variant<false, 256, 4, false>(w_down, w_down, h_rows, args, stream);
+}
+
+cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* sorted_ids, const int32_t* ntpp, int M, int top_k,
+                               int H, int cap, uint16_t* xg, cudaStream_t stream) {
+  gather_rows_kernel<<<(cap + 7) / 8, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), sorted_ids, ntpp,
+                                                        M * top_k, top_k, H / 8, cap, reinterpret_cast<uint4*>(xg));
+  return cudaGetLastError();
 }
 
 }  // namespace moe

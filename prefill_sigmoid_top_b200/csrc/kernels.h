@@ -40,9 +40,26 @@ struct GroupedGemmArgs {
 // `nmax` selects the token-tile width (32 or 128).  Tensor maps: a0/a1 are
 // the weight matrices viewed as 2-D [E*rows_per_expert, kdim]; b is x [M,H]
 // (up, row gather) or h [cap, I] (down, contiguous rows).
+// `gathered`: x_rows maps x already gathered into plan order ([cap, H],
+// 16-row boxes); otherwise x itself ([M, H], one-row boxes for tile::gather4).
 cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
-                              const GroupedGemmArgs& args, int nmax, cudaStream_t stream);
+                              const GroupedGemmArgs& args, int nmax, bool gathered, cudaStream_t stream);
+// xg[r] = x[sorted_ids[r] / top_k] for the real plan rows r < ntpp.
+cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* sorted_ids, const int32_t* ntpp, int M, int top_k,
+                               int H, int cap, uint16_t* xg, cudaStream_t stream);
 cudaError_t launch_grouped_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
                                 int nmax, cudaStream_t stream);
+
+// gemm_persistent.cu: one CTA per SM over a static tile list, 128-row token
+// tiles.  xg_rows / h_rows: plan-ordered [cap, kdim] tensors in 32-row boxes.
+// Weight tiles: up = 128 rows of gate and of up; down = 256 rows of W_down.
+// gather: x_rows maps x itself ([M,H], one-row boxes) and the kernel gathers
+// token rows with tile::gather4; otherwise x_rows is x in plan order.
+// deep_b: 4 weight stages + 5 token-row stages instead of 5 + 3.
+cudaError_t launch_persistent_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                                 const GroupedGemmArgs& args, int nmax, bool gather, bool deep_b, int num_sms,
+                                 cudaStream_t stream);
+cudaError_t launch_persistent_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
+                                   int nmax, bool deep_b, int num_sms, cudaStream_t stream);
 
 }  // namespace moe

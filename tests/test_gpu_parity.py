@@ -223,10 +223,23 @@ GEMM_CASES = [
 ]
 
 
-@pytest.mark.parametrize("nmax", ["32", "128"])
+GEMM_VARIANTS = [  # (token-tile width, x rows gathered in the GEMM or before it, persistent kernel)
+    ("32", "tma", "0"), ("32", "pregather", "0"), ("128", "tma", "0"), ("128", "pregather", "0"),
+    ("256", "tma", "0"), ("256", "pregather", "0"), ("128", "pregather", "1"), ("256", "pregather", "1"),
+    ("128", "tma", "1"), ("256", "tma", "1"),
+]
+
+
+@pytest.mark.parametrize("nmax,gather,persistent", GEMM_VARIANTS)
 @pytest.mark.parametrize("case", GEMM_CASES)
-def test_grouped_up_down(case, nmax, monkeypatch):
+@pytest.mark.parametrize("deep_b", ["0", "1"])
+def test_grouped_up_down(case, nmax, gather, persistent, deep_b, monkeypatch):
+    if deep_b == "1" and (persistent == "0" or nmax != "128"):
+        pytest.skip("the deep token ring exists for the persistent 128-row kernel only")
+    monkeypatch.setenv("MOE_PGEMM_DEEP_B", deep_b)
     monkeypatch.setenv("MOE_GEMM_NMAX", nmax)
+    monkeypatch.setenv("MOE_UP_GATHER", gather)
+    monkeypatch.setenv("MOE_GEMM_PERSISTENT", persistent)
     cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + case["E"], **case)
     d = to_dev(cfg)
     hb = host_bits(d)
