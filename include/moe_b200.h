@@ -214,6 +214,32 @@ MOE_API moe_status_t moe_prepare_nvfp4_weights(const uint8_t* codes, const uint8
                                        void* blob, size_t blob_bytes, moe_stream_t stream);
 MOE_API size_t moe_nvfp4_blob_bytes(moe_shape_t s, int which);
 
+/* ---------------------------------------------------------------- route, no allocation
+ * No counterpart on the pages: this entry point exists for callers that cannot
+ * allocate device memory themselves, for example a plugin running inside a
+ * host framework that owns every device allocation through its own pool, or a
+ * caller with a fixed, pre-budgeted memory footprint.  moe_route needs a
+ * caller-provided scratch buffer for the [M,E] fp32 router logits;
+ * moe_route_noalloc computes exactly the same routing (same kernels, same
+ * results) but keeps those logits in an array inside the library instead.
+ *  - Limit: M * E <= MOE_ROUTE_NOALLOC_MAX_LOGITS (4 MiB of fp32 logits, e.g.
+ *    M = 4096 tokens at E = 256); larger shapes return MOE_ERR_UNSUPPORTED
+ *    without launching anything.
+ *  - The array is a fixed 4 MiB device allocation made when the library is
+ *    loaded; every GPU the process uses holds one until the process exits.
+ *  - The first call on each device looks up the array's device address on
+ *    that device (the current device at the time of the call); that first
+ *    call should come before any stream capture on the device.
+ *  - All calls share the one array: calls whose kernels may overlap on the
+ *    GPU (other streams, other host threads) race and give wrong results, so
+ *    serialise them.  Nothing needs clearing between calls: each call writes
+ *    all M*E logits before it reads them.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Arguments, layouts and errors as moe_route, without ws / ws_bytes. */
+#define MOE_ROUTE_NOALLOC_MAX_LOGITS (1 << 20)
+MOE_API moe_status_t moe_route_noalloc(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                                       moe_shape_t s, int32_t* topk_ids, float* topk_w, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- errors -
  * Synchronises `stream`, reads the device error word and returns, in
  * *host_code, MOE_OK or the most severe device-detected status

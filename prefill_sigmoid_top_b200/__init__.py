@@ -99,6 +99,7 @@ def _declare(L):
         "moe_prepare_nvfp4_weights": (st, [vp, vp, _Shape, ctypes.c_int, vp, sz, vp]),
         "moe_nvfp4_blob_bytes": (sz, [_Shape, ctypes.c_int]),
         "moe_get_device_error": (st, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
+        "moe_route_noalloc": (st, [vp, vp, vp, _Shape, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

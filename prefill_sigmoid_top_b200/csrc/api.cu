@@ -241,6 +241,17 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
 
 }  // namespace
 
+namespace moe {
+int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,
+                     const void* topk_w) {
+  const moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!x || !w_router || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_status_string(moe_status_t st) {

@@ -6,7 +6,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "moe_b200.h"
+
 namespace moe {
+
+// api.cu: validation of moe_route's arguments (a moe_status_t value).
+int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,
+                     const void* topk_w);
 
 // router.cu
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,

@@ -16,6 +16,8 @@
 //  2. router_topk_kernel: one warp per token selects the K largest logits
 //     (descending; equal logits -> lower expert id) by K rounds of a warp
 //     argmax, then w_k = s_k / sum s with s = 1 / (1 + exp(-z)).
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -174,3 +176,49 @@ cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// moe_route_noalloc: moe_route for callers that cannot allocate device memory.
+// The [M,E] logits live in this fixed array instead of a caller workspace.
+// Device code could name the array directly; host code only has a host-side
+// stand-in for it, so the device address is looked up once per device (with
+// that device current) and passed to the kernels as a plain pointer.
+namespace {
+
+static __device__ __align__(256) float g_route_logits_scratch[MOE_ROUTE_NOALLOC_MAX_LOGITS];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+float* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device (set-up on first use).
+cudaError_t route_scratch_address(float** out) {
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    st = cudaGetSymbolAddress(&ptr, g_route_logits_scratch);
+    if (st != cudaSuccess) return st;
+    g_scratch_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_route_noalloc(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                                          moe_shape_t s, int32_t* topk_ids, float* topk_w, moe_stream_t stream) {
+  const int v = moe::check_route_args(s, x, w_router, topk_ids, topk_w);
+  if (v != MOE_OK) return static_cast<moe_status_t>(v);
+  if (static_cast<long long>(s.M) * s.E > MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ERR_UNSUPPORTED;
+  float* logits = nullptr;
+  if (route_scratch_address(&logits) != cudaSuccess) return MOE_ERR_CUDA;
+  auto cs = static_cast<cudaStream_t>(stream);
+  if (moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_router_topk(logits, s.M, s.E, s.top_k, topk_ids, topk_w, cs) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
