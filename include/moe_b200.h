@@ -37,7 +37,8 @@
  *    is set for status MOE_ERR_INVALID_INPUT or MOE_ERR_TIMEOUT.
  *  - Waits inside kernels are bounded (0.5 s each); on expiry the kernel
  *    sets the MOE_ERR_TIMEOUT bit and returns.
- *  - Accepted shapes: M >= 1; H % 256 == 0 and H <= 8192; I % 128 == 0;
+ *  - Accepted shapes: M >= 1; H % 256 == 0 and H <= 8192; I % 128 == 0
+ *    (I % 256 == 0 with MOE_W_NVFP4 weights);
  *    1 <= top_k <= min(E, 32); 1 <= E <= 1024; block_size a power of two in
  *    [16, 256]; M * top_k < 2^31.  Others return MOE_ERR_UNSUPPORTED.
  */
@@ -80,8 +81,10 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_NVFP4 = 1 } moe_wdtype_t;
 /* Expert weights.
  * MOE_W_BF16:  gate, up: bf16 [E, I, H]; down: bf16 [E, H, I] (the contraction
  *              dimension is contiguous); the *_gs pointers are ignored.
- * MOE_W_NVFP4: gate, up, down: blobs written by moe_quantize_nvfp4_weights;
- *              gate_gs, up_gs, down_gs: device fp32 [E] per-expert global scales. */
+ * MOE_W_NVFP4: gate, up, down: blobs written by moe_prepare_nvfp4_weights
+ *              (from moe_quantize_nvfp4 of W_gate/W_up as E matrices [I,H] and
+ *              W_down as E matrices [H,I]); gate_gs, up_gs, down_gs: the device
+ *              fp32 [E] per-expert global scales that moe_quantize_nvfp4 wrote. */
 typedef struct {
   moe_wdtype_t dtype;
   const void* gate;
@@ -143,7 +146,9 @@ MOE_API size_t moe_align_capacity(moe_shape_t s); /* M*top_k + E*(block_size-1) 
  * ws (nullable): moe_up_workspace_size(s, dtype) bytes of device scratch.  With
  * it, wide token tiles first gather x into plan order there and read it as
  * contiguous rows; without it the rows are gathered inside the GEMM.  Both
- * give the same result.  MOE_W_NVFP4 quantises x on the fly into ws. */
+ * give the same result.  MOE_W_NVFP4: x is quantised on the fly (global scale
+ * from the amax over all of x) into ws (required), and the accumulators are
+ * scaled by gs_gate[e] * gs_x and gs_up[e] * gs_x before SwiGLU. */
 MOE_API moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
                                    moe_shape_t s, moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err_flag,
                                    moe_stream_t stream);
@@ -154,7 +159,9 @@ MOE_API size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype);
  * non-padding plan row r of expert e, with f = sorted_ids[r]:
  *   y[f, :] = bf16(h[r] . w.down[e]^T)   (fp32 accumulation)
  * h: bf16 [cap, I]; y: bf16 [M*top_k, H] (slot-major: y[t, k, :]).
- * MOE_W_NVFP4 quantises h on the fly into ws. */
+ * MOE_W_NVFP4: h is quantised on the fly (global scale from the amax over the
+ * real plan rows of h) into ws, moe_down_workspace_size(s, MOE_W_NVFP4) bytes
+ * (required); the accumulators are scaled by gs_down[e] * gs_h. */
 MOE_API moe_status_t moe_grouped_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
                               moe_shape_t s, moe_bf16_t* y, void* ws, size_t ws_bytes, int32_t* err_flag,
                               moe_stream_t stream);
@@ -209,7 +216,11 @@ MOE_API size_t moe_nvfp4_quantize_workspace_size(int64_t n_mats);
 
 /* Repack quantised expert weights (codes/scales as written by
  * moe_quantize_nvfp4 for all E experts of one projection) into the blob the
- * grouped kernels read.  which: 0 gate, 1 up, 2 down. */
+ * grouped kernels read: the codes unchanged, then the scales regrouped into
+ * 512-byte atoms of 128 rows x 64 columns (row r, column block j at byte
+ * (r%32)*16 + ((r%128)/32)*4 + j%4 of atom [r/128][j/4]), the layout the
+ * block-scaled tensor-core MMA takes its scale factors in.
+ * which: 0 gate, 1 up, 2 down; blob: moe_nvfp4_blob_bytes(s, which) bytes. */
 MOE_API moe_status_t moe_prepare_nvfp4_weights(const uint8_t* codes, const uint8_t* scales, moe_shape_t s, int which,
                                        void* blob, size_t blob_bytes, moe_stream_t stream);
 MOE_API size_t moe_nvfp4_blob_bytes(moe_shape_t s, int which);

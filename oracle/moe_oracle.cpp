@@ -508,7 +508,27 @@ void oracle_nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_
 // Activations: x is quantised from bf16 with gs from amax over all of x;
 // h (after bf16 rounding) is quantised with gs from amax over all M*K slot
 // rows of the call, so this computes h for every token, then y and out for
-// the chosen tokens.  Returns 3 if a needed expert is missing.
+// the chosen tokens.  Work is grouped by expert so that each expert matrix is
+// dequantised once.  Returns 3 if a needed expert is missing.
+namespace {
+struct Fp4Tables {
+  double e2m1[16];
+  double e4m3[256];
+  Fp4Tables() {
+    for (int c = 0; c < 16; ++c) e2m1[c] = e2m1_value(static_cast<uint8_t>(c));
+    for (int c = 0; c < 256; ++c) e4m3[c] = e4m3_value(static_cast<uint8_t>(c));
+  }
+};
+
+void dequantize_matrix(const Fp4Tables& T, const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                       float gs, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c)
+      out[r * cols + c] = T.e2m1[codes[r * cols + c]] * T.e4m3[scales[r * (cols / 16) + c / 16]] * static_cast<double>(gs);
+}
+}  // namespace
+
 int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float* bias,
                        const uint8_t* const* gate_codes, const uint8_t* const* gate_scales, const float* gate_gs,
                        const uint8_t* const* up_codes, const uint8_t* const* up_scales, const float* up_gs,
@@ -517,11 +537,13 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
                        const int32_t* tokens, int n_tokens, int32_t* topk_ids_all, double* topk_w_all,
                        uint16_t* h_all, uint16_t* y_out, uint16_t* out, uint16_t* residual_out,
                        double* out64, double* s64) {
+  static const Fp4Tables T;
   // routing for every token (h needs all of them)
   std::vector<float> z(static_cast<size_t>(M) * E);
   oracle_router_logits(x, w_router, bias, M, H, E, z.data(), nullptr);
   oracle_topk(z.data(), M, E, K, topk_ids_all, topk_w_all);
-  for (int64_t s = 0; s < static_cast<int64_t>(M) * K; ++s) {
+  const int64_t n_slots = static_cast<int64_t>(M) * K;
+  for (int64_t s = 0; s < n_slots; ++s) {
     const int e = topk_ids_all[s];
     if (!gate_codes[e] || !up_codes[e] || !gate_scales[e] || !up_scales[e]) return 3;
   }
@@ -530,7 +552,7 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
       const int e = topk_ids_all[static_cast<size_t>(tokens[i]) * K + k];
       if (!down_codes[e] || !down_scales[e]) return 3;
     }
-  // x -> NVFP4 (gs over all of x)
+  // x -> NVFP4 (gs over all of x), dequantised
   std::vector<float> xf(static_cast<size_t>(M) * H);
   float xamax = 0.0f;
   for (size_t i = 0; i < xf.size(); ++i) {
@@ -540,19 +562,26 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
   const float xgs = oracle_nvfp4_global_scale(xamax);
   std::vector<uint8_t> xc(xf.size()), xs(xf.size() / 16);
   oracle_nvfp4_quantize(xf.data(), M, H, xgs, xc.data(), xs.data());
-  // h for every slot
-  const int64_t n_slots = static_cast<int64_t>(M) * K;
+  std::vector<double> xd(xf.size());
+  dequantize_matrix(T, xc.data(), xs.data(), M, H, xgs, xd.data());
+  // h for every slot, expert by expert
+  std::vector<std::vector<int64_t>> by_expert(E);
+  for (int64_t s = 0; s < n_slots; ++s) by_expert[topk_ids_all[s]].push_back(s);
+  std::vector<double> wg(static_cast<size_t>(I) * H), wu(static_cast<size_t>(I) * H);
+  for (int e = 0; e < E; ++e) {
+    if (by_expert[e].empty()) continue;
+    dequantize_matrix(T, gate_codes[e], gate_scales[e], I, H, gate_gs[e], wg.data());
+    dequantize_matrix(T, up_codes[e], up_scales[e], I, H, up_gs[e], wu.data());
+    const int64_t ns = static_cast<int64_t>(by_expert[e].size());
 #pragma omp parallel for schedule(dynamic)
-  for (int64_t s = 0; s < n_slots; ++s) {
-    const int64_t t = s / K;
-    const int e = topk_ids_all[s];
-    std::vector<double> xd(H);
-    for (int c = 0; c < H; ++c) xd[c] = oracle_nvfp4_value(xc.data(), xs.data(), H, xgs, t, c);
-    for (int i = 0; i < I; ++i) {
+    for (int64_t j = 0; j < ns * I; ++j) {
+      const int64_t s = by_expert[e][j / I];
+      const int i = static_cast<int>(j % I);
+      const double* xr = xd.data() + (s / K) * H;
       double g = 0.0, u = 0.0;
       for (int c = 0; c < H; ++c) {
-        g += xd[c] * oracle_nvfp4_value(gate_codes[e], gate_scales[e], H, gate_gs[e], i, c);
-        u += xd[c] * oracle_nvfp4_value(up_codes[e], up_scales[e], H, up_gs[e], i, c);
+        g += xr[c] * wg[static_cast<size_t>(i) * H + c];
+        u += xr[c] * wu[static_cast<size_t>(i) * H + c];
       }
       h_all[s * I + i] = bf16_round(g * sigmoid(g) * u);
     }
@@ -561,28 +590,36 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
   float hamax = 0.0f;
   for (int64_t i = 0; i < n_slots * I; ++i) hamax = std::max(hamax, std::fabs(bf16_value_f(h_all[i])));
   const float hgs = oracle_nvfp4_global_scale(hamax);
-  // y for the chosen tokens
+  // y for the chosen tokens, expert by expert
   std::vector<uint16_t> y_local;
   uint16_t* y = y_out;
   if (!y) {
     y_local.resize(static_cast<size_t>(n_tokens) * K * H);
     y = y_local.data();
   }
-#pragma omp parallel for schedule(dynamic)
-  for (int s = 0; s < n_tokens * K; ++s) {
-    const int i = s / K, k = s % K;
-    const int64_t slot = static_cast<int64_t>(tokens[i]) * K + k;
-    const int e = topk_ids_all[slot];
-    std::vector<float> hf(I);
-    for (int c = 0; c < I; ++c) hf[c] = bf16_value_f(h_all[slot * I + c]);
-    std::vector<uint8_t> hc(I), hs(I / 16);
-    oracle_nvfp4_quantize(hf.data(), 1, I, hgs, hc.data(), hs.data());
-    std::vector<double> hd(I);
-    for (int c = 0; c < I; ++c) hd[c] = oracle_nvfp4_value(hc.data(), hs.data(), I, hgs, 0, c);
-    for (int r = 0; r < H; ++r) {
-      double acc = 0.0;
-      for (int c = 0; c < I; ++c) acc += hd[c] * oracle_nvfp4_value(down_codes[e], down_scales[e], I, down_gs[e], r, c);
-      y[static_cast<size_t>(s) * H + r] = bf16_round(acc);
+  std::vector<std::vector<int>> chosen_by_expert(E);  // local slot index i*K + k
+  for (int i = 0; i < n_tokens; ++i)
+    for (int k = 0; k < K; ++k)
+      chosen_by_expert[topk_ids_all[static_cast<size_t>(tokens[i]) * K + k]].push_back(i * K + k);
+  std::vector<double> wd(static_cast<size_t>(H) * I);
+  for (int e = 0; e < E; ++e) {
+    if (chosen_by_expert[e].empty()) continue;
+    dequantize_matrix(T, down_codes[e], down_scales[e], H, I, down_gs[e], wd.data());
+    for (int ls : chosen_by_expert[e]) {
+      const int i = ls / K, k = ls % K;
+      const int64_t slot = static_cast<int64_t>(tokens[i]) * K + k;
+      std::vector<float> hf(I);
+      for (int c = 0; c < I; ++c) hf[c] = bf16_value_f(h_all[slot * I + c]);
+      std::vector<uint8_t> hc(I), hs(I / 16);
+      oracle_nvfp4_quantize(hf.data(), 1, I, hgs, hc.data(), hs.data());
+      std::vector<double> hd(I);
+      dequantize_matrix(T, hc.data(), hs.data(), 1, I, hgs, hd.data());
+#pragma omp parallel for schedule(static)
+      for (int r = 0; r < H; ++r) {
+        double acc = 0.0;
+        for (int c = 0; c < I; ++c) acc += hd[c] * wd[static_cast<size_t>(r) * I + c];
+        y[static_cast<size_t>(ls) * H + r] = bf16_round(acc);
+      }
     }
   }
   if (out) {

@@ -18,7 +18,9 @@ import torch
 __all__ = [
     "MoEError", "Shape", "library", "route", "align_block_size", "grouped_up_swiglu", "grouped_down",
     "finalize_rmsnorm", "layer", "layer_workspace_size", "up_workspace_size", "layer_workspace_layout", "align_capacity",
-    "route_workspace_size", "get_device_error", "status_string", "STATUS",
+    "route_workspace_size", "get_device_error", "status_string", "STATUS", "NVFP4Weights", "quantize_nvfp4",
+    "prepare_nvfp4_weights", "nvfp4_weights", "nvfp4_blob_bytes", "grouped_up_swiglu_nvfp4", "grouped_down_nvfp4",
+    "layer_nvfp4", "down_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -280,6 +282,108 @@ def layer(x, w_router, bias, w_gate, w_up, w_down, gamma, eps, top_k, block_size
     if out is None:
         out = torch.empty_like(x)
     w = _weights_struct(w_gate, w_up, w_down)
+    _check(library().moe_layer(_ptr(_bf16(x)), _ptr(_bf16(w_router)), _ptr(bias), ctypes.byref(w),
+                               _ptr(_bf16(gamma)), float(eps), shape.c(), _ptr(out), _ptr(residual_out),
+                               _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_layer")
+    return out
+
+
+# ------------------------------------------------------------------ NVFP4
+@dataclass
+class NVFP4Weights:
+    """Prepared NVFP4 expert weights: one blob (uint8) per projection and the
+    per-expert fp32 global scales."""
+    gate: torch.Tensor
+    up: torch.Tensor
+    down: torch.Tensor
+    gate_gs: torch.Tensor
+    up_gs: torch.Tensor
+    down_gs: torch.Tensor
+
+    def c(self) -> _Weights:
+        return _Weights(MOE_W_NVFP4, self.gate.data_ptr(), self.up.data_ptr(), self.down.data_ptr(),
+                        self.gate_gs.data_ptr(), self.up_gs.data_ptr(), self.down_gs.data_ptr())
+
+
+def quantize_nvfp4(w):
+    """w bf16 [n_mats, rows, cols] -> (codes uint8 [n,rows,cols/2], scales uint8 [n,rows,cols/16], gs fp32 [n])."""
+    _need_cuda(w)
+    n, rows, cols = w.shape
+    codes = torch.empty(n, rows, cols // 2, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(n, rows, cols // 16, dtype=torch.uint8, device=w.device)
+    gs = torch.empty(n, dtype=torch.float32, device=w.device)
+    ws = torch.empty(int(library().moe_nvfp4_quantize_workspace_size(n)), dtype=torch.uint8, device=w.device)
+    _check(library().moe_quantize_nvfp4(_ptr(_bf16(w)), n, rows, cols, _ptr(codes), _ptr(scales), _ptr(gs), _ptr(ws),
+                                        ws.numel(), _stream()), "moe_quantize_nvfp4")
+    return codes, scales, gs
+
+
+def nvfp4_blob_bytes(shape: Shape, which: int) -> int:
+    return int(library().moe_nvfp4_blob_bytes(shape.c(), which))
+
+
+def prepare_nvfp4_weights(codes, scales, shape: Shape, which: int):
+    blob = torch.empty(nvfp4_blob_bytes(shape, which), dtype=torch.uint8, device=codes.device)
+    _check(library().moe_prepare_nvfp4_weights(_ptr(codes), _ptr(scales), shape.c(), which, _ptr(blob), blob.numel(),
+                                               _stream()), "moe_prepare_nvfp4_weights")
+    return blob
+
+
+def nvfp4_weights(w_gate, w_up, w_down, shape: Shape) -> NVFP4Weights:
+    """Quantise bf16 expert weights and prepare the blobs the NVFP4 kernels read."""
+    blobs, gss = [], []
+    for which, w in enumerate((w_gate, w_up, w_down)):
+        codes, scales, gs = quantize_nvfp4(w)
+        blobs.append(prepare_nvfp4_weights(codes, scales, shape, which))
+        gss.append(gs)
+        del codes, scales
+    return NVFP4Weights(blobs[0], blobs[1], blobs[2], gss[0], gss[1], gss[2])
+
+
+def down_workspace_size(shape: Shape, wdtype: int = MOE_W_BF16) -> int:
+    return int(library().moe_down_workspace_size(shape.c(), wdtype))
+
+
+def grouped_up_swiglu_nvfp4(x, nw: NVFP4Weights, plan, shape: Shape, h=None, err_flag=None, ws=None):
+    """NVFP4 form of grouped_up_swiglu (x quantised on the fly into ws)."""
+    _need_cuda(x)
+    if h is None:
+        h = torch.empty(align_capacity(shape), shape.I, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = torch.empty(up_workspace_size(shape, MOE_W_NVFP4), dtype=torch.uint8, device=x.device)
+    w = nw.c()
+    p = _plan_struct(plan)
+    _check(library().moe_grouped_up_swiglu(_ptr(_bf16(x)), ctypes.byref(w), ctypes.byref(p), shape.c(), _ptr(h),
+                                           _ptr(ws), ws.numel(), _ptr(err_flag), _stream()), "moe_grouped_up_swiglu")
+    return h
+
+
+def grouped_down_nvfp4(h, nw: NVFP4Weights, plan, shape: Shape, y=None, err_flag=None, ws=None):
+    """NVFP4 form of grouped_down (h quantised on the fly into ws)."""
+    _need_cuda(h)
+    if y is None:
+        y = torch.empty(shape.M * shape.top_k, shape.H, dtype=torch.bfloat16, device=h.device)
+    if ws is None:
+        ws = torch.empty(down_workspace_size(shape, MOE_W_NVFP4), dtype=torch.uint8, device=h.device)
+    w = nw.c()
+    p = _plan_struct(plan)
+    _check(library().moe_grouped_down(_ptr(_bf16(h)), ctypes.byref(w), ctypes.byref(p), shape.c(), _ptr(y), _ptr(ws),
+                                      ws.numel(), _ptr(err_flag), _stream()), "moe_grouped_down")
+    return y
+
+
+def layer_nvfp4(x, w_router, bias, nw: NVFP4Weights, gamma, eps, top_k, block_size, I, ws=None, out=None,
+                residual_out=None, topk_ids=None, topk_w=None):
+    """The whole layer with NVFP4 expert weights; returns out [M,H] bf16."""
+    _need_cuda(x, w_router, gamma)
+    M, H = x.shape
+    E = w_router.shape[0]
+    shape = Shape(M, H, I, E, top_k, block_size)
+    if ws is None:
+        ws = torch.empty(layer_workspace_size(shape, MOE_W_NVFP4), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    w = nw.c()
     _check(library().moe_layer(_ptr(_bf16(x)), _ptr(_bf16(w_router)), _ptr(bias), ctypes.byref(w),
                                _ptr(_bf16(gamma)), float(eps), shape.c(), _ptr(out), _ptr(residual_out),
                                _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_layer")

@@ -67,6 +67,21 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
+// 2-D byte tensor [rows, cols_bytes] read in boxes of box_rows x 128 bytes
+// with the 128-byte swizzle (packed e2m1 codes: 256 elements per box row).
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols_bytes, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols_bytes, rows};
+  cuuint64_t strides[1] = {cols_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Token-tile width of the grouped kernels, from the mean routed rows per
 // expert (known on the host without reading the plan back): decode shapes
 // (<= 24) use 32-row tiles, larger ones 128-row tiles.  256-row tiles measured
@@ -101,6 +116,36 @@ bool want_pregather(const moe_shape_t& s) {
 }
 
 size_t pregather_bytes(const moe_shape_t& s) { return align_up(cap_rows(s) * s.H * sizeof(uint16_t)); }
+
+// ---------------------------------------------------------------- NVFP4 sizes
+// Upper bound on 128-row token tiles (sum over experts of ceil(count/128)).
+int nvfp4_tiles_ub(const moe_shape_t& s) {
+  const long long mk = static_cast<long long>(s.M) * s.top_k;
+  return static_cast<int>(mk / 128 + (mk < s.E ? mk : s.E));
+}
+// Tile-aligned NVFP4 activation copy of `cols`-wide rows: amax word, codes, scale atoms.
+struct ActLayout {
+  size_t amax, codes, atoms, total;
+};
+ActLayout act_layout(const moe_shape_t& s, int cols) {
+  ActLayout L{};
+  const size_t rows = static_cast<size_t>(nvfp4_tiles_ub(s)) * 128;
+  L.amax = 0;
+  L.codes = kAlign;
+  L.atoms = align_up(L.codes + rows * cols / 2);
+  L.total = align_up(L.atoms + static_cast<size_t>(nvfp4_tiles_ub(s)) * (cols / 64) * 512);
+  return L;
+}
+// Blob of one projection: codes [rows, cols/2] then scale atoms.
+void blob_dims(const moe_shape_t& s, int which, int64_t* rows, int64_t* cols) {
+  *rows = static_cast<int64_t>(s.E) * (which == 2 ? s.H : s.I);
+  *cols = which == 2 ? s.I : s.H;
+}
+size_t blob_codes_bytes(const moe_shape_t& s, int which) {
+  int64_t r, c;
+  blob_dims(s, which, &r, &c);
+  return static_cast<size_t>(r) * c / 2;
+}
 
 // Whether the batch/prefill shapes run the persistent kernel (one CTA per SM,
 // deep weight ring, double-buffered accumulators).  MOE_GEMM_PERSISTENT=0|1
@@ -143,6 +188,22 @@ moe_status_t check_bf16_weights(const moe_weights_t* w) {
   if (w->dtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
+
+moe_status_t check_weights(const moe_weights_t* w, const moe_shape_t& s) {
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (w->dtype != MOE_W_BF16 && w->dtype != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+  if (w->dtype == MOE_W_NVFP4) {
+    if (!w->gate_gs || !w->up_gs || !w->down_gs) return MOE_ERR_INVALID_ARG;
+    if (s.I % 256 != 0) return MOE_ERR_UNSUPPORTED;  // the NVFP4 kernels step 256 elements along I
+  }
+  return MOE_OK;
+}
+
+// NVFP4 up: amax of x -> tile-aligned NVFP4 copy of the routed x rows -> block-scaled GEMM.
+moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
+                          const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream);
+moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
+                            const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream);
 
 moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
                     moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t stream) {
@@ -205,8 +266,84 @@ moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_pla
   return cuda_status(moe::launch_grouped_down(md, mh, a, choose_nmax(s), stream));
 }
 
+int num_sms();
+
+moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
+                          const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream) {
+  const ActLayout L = act_layout(s, s.H);
+  auto* base = static_cast<uint8_t*>(ws);
+  auto* amax = reinterpret_cast<unsigned*>(base + L.amax);
+  const int tiles = nvfp4_tiles_ub(s);
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_amax_all(x, static_cast<int64_t>(s.M) * s.H, amax, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_quantize_tiles(x, true, plan->sorted_ids, plan->expert_counts, plan->expert_offsets, s.E, s.top_k,
+                                 s.M * s.top_k, s.H, tiles, amax, base + L.codes, base + L.atoms, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  CUtensorMap mg, mu, mx;
+  const uint64_t wrows = static_cast<uint64_t>(s.E) * s.I;
+  if (!make_map_u8(&mg, w->gate, wrows, s.H / 2, 128) || !make_map_u8(&mu, w->up, wrows, s.H / 2, 128) ||
+      !make_map_u8(&mx, base + L.codes, static_cast<uint64_t>(tiles) * 128, s.H / 2, 32))
+    return MOE_ERR_CUDA;
+  moe::Nvfp4GemmArgs a{};
+  a.g.sorted_ids = plan->sorted_ids;
+  a.g.expert_counts = plan->expert_counts;
+  a.g.expert_offsets = plan->expert_offsets;
+  a.g.out = h;
+  a.g.err = err;
+  a.g.M = s.M;
+  a.g.E = s.E;
+  a.g.top_k = s.top_k;
+  a.g.rows_per_expert = s.I;
+  a.g.kdim = s.H;
+  a.g.out_ld = s.I;
+  a.sfa0 = static_cast<const uint8_t*>(w->gate) + blob_codes_bytes(s, 0);
+  a.sfa1 = static_cast<const uint8_t*>(w->up) + blob_codes_bytes(s, 1);
+  a.sfb = base + L.atoms;
+  a.gs_a0 = w->gate_gs;
+  a.gs_a1 = w->up_gs;
+  a.act_amax = amax;
+  return cuda_status(moe::launch_nvfp4_up(mg, mu, mx, a, num_sms(), stream));
+}
+
+moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
+                            const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream) {
+  const ActLayout L = act_layout(s, s.I);
+  auto* base = static_cast<uint8_t*>(ws);
+  auto* amax = reinterpret_cast<unsigned*>(base + L.amax);
+  const int tiles = nvfp4_tiles_ub(s);
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_amax_plan_rows(h, plan->sorted_ids, plan->num_tokens_post_padded, s.M * s.top_k, s.I,
+                                 static_cast<int>(cap_rows(s)), amax, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::launch_quantize_tiles(h, false, plan->sorted_ids, plan->expert_counts, plan->expert_offsets, s.E, s.top_k,
+                                 s.M * s.top_k, s.I, tiles, amax, base + L.codes, base + L.atoms, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  CUtensorMap md, mh;
+  if (!make_map_u8(&md, w->down, static_cast<uint64_t>(s.E) * s.H, s.I / 2, 128) ||
+      !make_map_u8(&mh, base + L.codes, static_cast<uint64_t>(tiles) * 128, s.I / 2, 32))
+    return MOE_ERR_CUDA;
+  moe::Nvfp4GemmArgs a{};
+  a.g.sorted_ids = plan->sorted_ids;
+  a.g.expert_counts = plan->expert_counts;
+  a.g.expert_offsets = plan->expert_offsets;
+  a.g.out = y;
+  a.g.err = err;
+  a.g.M = s.M;
+  a.g.E = s.E;
+  a.g.top_k = s.top_k;
+  a.g.rows_per_expert = s.H;
+  a.g.kdim = s.I;
+  a.g.out_ld = s.H;
+  a.sfa0 = static_cast<const uint8_t*>(w->down) + blob_codes_bytes(s, 2);
+  a.sfa1 = a.sfa0;
+  a.sfb = base + L.atoms;
+  a.gs_a0 = w->down_gs;
+  a.gs_a1 = w->down_gs;
+  a.act_amax = amax;
+  return cuda_status(moe::launch_nvfp4_down(md, mh, a, num_sms(), stream));
+}
+
 moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
-  (void)dt;
   moe_layer_ws_layout_t L{};
   const size_t mk = static_cast<size_t>(s.M) * s.top_k;
   const size_t cap = cap_rows(s);
@@ -233,8 +370,11 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   off = align_up(off + cap * s.I * sizeof(uint16_t));
   L.y = off;
   off = align_up(off + mk * s.H * sizeof(uint16_t));
-  L.act_scratch = off;  // x gathered into plan order (up projection)
-  off = align_up(off + pregather_bytes(s));
+  L.act_scratch = off;  // bf16: x gathered into plan order; NVFP4: the two tile-aligned activation copies
+  if (dt == MOE_W_NVFP4)
+    off = align_up(off + act_layout(s, s.H).total + act_layout(s, s.I).total);
+  else
+    off = align_up(off + pregather_bytes(s));
   L.total = off;
   return L;
 }
@@ -279,13 +419,13 @@ size_t moe_route_workspace_size(moe_shape_t s) {
 
 size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK) return 0;
-  (void)dtype;
+  if (dtype == MOE_W_NVFP4) return act_layout(s, s.H).total;
   return (want_pregather(s) || want_persistent(s)) ? pregather_bytes(s) : 0;
 }
 
 size_t moe_down_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK) return 0;
-  return dtype == MOE_W_BF16 ? 0 : 0;
+  return dtype == MOE_W_NVFP4 ? act_layout(s, s.I).total : 0;
 }
 
 moe_status_t moe_route(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, moe_shape_t s,
@@ -319,23 +459,31 @@ moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, 
                                    moe_stream_t stream) {
   moe_status_t st = check_shape(s);
   if (st != MOE_OK) return st;
-  if ((st = check_bf16_weights(w)) != MOE_OK) return st;
+  if ((st = check_weights(w, s)) != MOE_OK) return st;
   if ((st = check_plan(plan)) != MOE_OK) return st;
   if (!x || !h || !w->gate || !w->up) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(h) || !aligned16(w->gate) || !aligned16(w->up)) return MOE_ERR_INVALID_ARG;
+  if (w->dtype == MOE_W_NVFP4) {
+    if (!ws || ws_bytes < moe_up_workspace_size(s, MOE_W_NVFP4) || !aligned16(ws) || !plan->num_tokens_post_padded)
+      return MOE_ERR_WORKSPACE;
+    return run_up_nvfp4(x, w, plan, s, h, ws, err_flag, static_cast<cudaStream_t>(stream));
+  }
   return run_up(x, w, plan, s, h, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_grouped_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, moe_shape_t s,
                               moe_bf16_t* y, void* ws, size_t ws_bytes, int32_t* err_flag, moe_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   moe_status_t st = check_shape(s);
   if (st != MOE_OK) return st;
-  if ((st = check_bf16_weights(w)) != MOE_OK) return st;
+  if ((st = check_weights(w, s)) != MOE_OK) return st;
   if ((st = check_plan(plan)) != MOE_OK) return st;
   if (!h || !y || !w->down) return MOE_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(y) || !aligned16(w->down)) return MOE_ERR_INVALID_ARG;
+  if (w->dtype == MOE_W_NVFP4) {
+    if (!ws || ws_bytes < moe_down_workspace_size(s, MOE_W_NVFP4) || !aligned16(ws) || !plan->num_tokens_post_padded)
+      return MOE_ERR_WORKSPACE;
+    return run_down_nvfp4(h, w, plan, s, y, ws, err_flag, static_cast<cudaStream_t>(stream));
+  }
   return run_down(h, w, plan, s, y, err_flag, static_cast<cudaStream_t>(stream));
 }
 
@@ -372,7 +520,7 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   moe_status_t st = check_shape(s);
   if (st != MOE_OK) return st;
   if (!w) return MOE_ERR_INVALID_ARG;
-  if ((st = check_bf16_weights(w)) != MOE_OK) return st;
+  if ((st = check_weights(w, s)) != MOE_OK) return st;
   if (!x || !w_router || !gamma || !out || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(gamma) || !aligned16(out) || !aligned16(w->gate) ||
       !aligned16(w->up) || !aligned16(w->down) || (residual_out && !aligned16(residual_out)))
@@ -402,30 +550,52 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
                                           err, cs))) != MOE_OK)
     return st;
   moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
-  if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
-  if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
+  if (w->dtype == MOE_W_NVFP4) {
+    uint8_t* act = base + L.act_scratch;
+    if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs)) != MOE_OK) return st;
+    if ((st = run_down_nvfp4(h, w, &plan, s, y, act + act_layout(s, s.H).total, err, cs)) != MOE_OK) return st;
+  } else {
+    if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
+    if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
+  }
   return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
 }
 
 moe_status_t moe_quantize_nvfp4(const moe_bf16_t* src, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* codes,
                                 uint8_t* scales, float* gs, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  (void)src; (void)n_mats; (void)rows; (void)cols; (void)codes; (void)scales; (void)gs; (void)ws; (void)ws_bytes;
-  (void)stream;
-  return MOE_ERR_UNSUPPORTED;
+  if (n_mats < 1 || rows < 1 || cols < 16 || cols % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!src || !codes || !scales || !gs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(codes) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_nvfp4_quantize_workspace_size(n_mats) || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  return cuda_status(moe::launch_nvfp4_quantize(src, n_mats, rows, cols, codes, scales, gs,
+                                                static_cast<unsigned*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
-size_t moe_nvfp4_quantize_workspace_size(int64_t n_mats) { return align_up(static_cast<size_t>(n_mats) * 4); }
+size_t moe_nvfp4_quantize_workspace_size(int64_t n_mats) {
+  return n_mats < 1 ? 0 : align_up(static_cast<size_t>(n_mats) * 4);
+}
 
 moe_status_t moe_prepare_nvfp4_weights(const uint8_t* codes, const uint8_t* scales, moe_shape_t s, int which,
                                        void* blob, size_t blob_bytes, moe_stream_t stream) {
-  (void)codes; (void)scales; (void)s; (void)which; (void)blob; (void)blob_bytes; (void)stream;
-  return MOE_ERR_UNSUPPORTED;
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (which < 0 || which > 2) return MOE_ERR_INVALID_ARG;
+  if (!codes || !scales || !blob || !aligned16(codes) || !aligned16(blob)) return MOE_ERR_INVALID_ARG;
+  if (blob_bytes < moe_nvfp4_blob_bytes(s, which)) return MOE_ERR_WORKSPACE;
+  int64_t rows, cols;
+  blob_dims(s, which, &rows, &cols);
+  auto cs = static_cast<cudaStream_t>(stream);
+  auto* b = static_cast<uint8_t*>(blob);
+  if (cudaMemcpyAsync(b, codes, static_cast<size_t>(rows) * cols / 2, cudaMemcpyDeviceToDevice, cs) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(moe::launch_nvfp4_scales_to_atoms(scales, rows, cols, b + blob_codes_bytes(s, which), cs));
 }
 
 size_t moe_nvfp4_blob_bytes(moe_shape_t s, int which) {
-  (void)s;
-  (void)which;
-  return 0;
+  if (check_shape(s) != MOE_OK || which < 0 || which > 2) return 0;
+  int64_t rows, cols;
+  blob_dims(s, which, &rows, &cols);
+  return static_cast<size_t>(rows) * cols / 2 + static_cast<size_t>(rows) * cols / 16;
 }
 
 moe_status_t moe_get_device_error(const int32_t* err_flag, moe_stream_t stream, int32_t* host_code) {

@@ -111,6 +111,14 @@ __device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (both 16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -186,6 +194,41 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte block stored contiguously
+// (no swizzle; core matrices of 8 rows x 16 bytes, 128 bytes apart): the
+// source form of tcgen05.cp ... 32x128b.
+__device__ __forceinline__ uint64_t smem_desc_32x16B(const void* p) {
+  const uint64_t addr = (smem_addr(p) & 0x3FFFFu) >> 4;
+  return addr | (uint64_t(1) << 16) | (uint64_t(128 >> 4) << 32) | (uint64_t(1) << 46);
+}
+
+// Copy a 32-row x 16-byte block from shared memory into tensor memory at
+// `taddr` (32 lanes x 4 columns), replicated into all four lane quarters.
+__device__ __forceinline__ void tmem_copy_32x16B_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor for kind::mxf4nvf4 (e2m1 A and B, per-16 e4m3 block
+// scales, fp32 accumulate), K-major, M = 128: A format (1 = e2m1) at [7,10),
+// B format at [10,13), N >> 3 at [17,23), scale format 0 (e4m3) at bit 23,
+// M >> 4 at [24,29); scale-factor ids and the K size bit are 0.
+__host__ __device__ constexpr uint32_t umma_idesc_nvfp4(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D[tmem] (+)= (A * sfa) * (B * sfb)^T, K = 64 e2m1 elements, block-16 scales
+// read from tensor memory at sfa / sfb.
+__device__ __forceinline__ void umma_nvfp4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
 

@@ -68,4 +68,33 @@ cudaError_t launch_persistent_up(const CUtensorMap& w_gate, const CUtensorMap& w
 cudaError_t launch_persistent_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
                                    int nmax, bool deep_b, int num_sms, cudaStream_t stream);
 
+// nvfp4.cu ------------------------------------------------------------------
+struct Nvfp4GemmArgs {
+  GroupedGemmArgs g;      // kdim in elements; out / plan / shape as for bf16
+  const uint8_t* sfa0;    // weight scale atoms of the tm_a0 rows ([rows/128][kdim/64][512])
+  const uint8_t* sfa1;    // of the tm_a1 rows (up: W_up; down: W_down again)
+  const uint8_t* sfb;     // activation scale atoms, tile-aligned ([tiles][kdim/64][512])
+  const float* gs_a0;     // [E] global scales of the tm_a0 matrix
+  const float* gs_a1;     // [E]
+  const unsigned* act_amax;  // activation amax (fp32 bits); gs = amax / 2688
+};
+
+// Quantise n_mats matrices [rows, cols] (bf16, back to back) to NVFP4 codes /
+// row-major e4m3 scales / per-matrix global scales; amax_bits: n_mats words.
+cudaError_t launch_nvfp4_quantize(const uint16_t* src, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* codes,
+                                  uint8_t* scales, float* gs, unsigned* amax_bits, cudaStream_t stream);
+cudaError_t launch_nvfp4_scales_to_atoms(const uint8_t* scales, int64_t rows, int64_t cols, uint8_t* atoms,
+                                         cudaStream_t stream);
+// *amax_bits = max(*amax_bits, max |src[0..n)|) (bits of a non-negative float).
+cudaError_t launch_amax_all(const uint16_t* src, int64_t n, unsigned* amax_bits, cudaStream_t stream);
+cudaError_t launch_amax_plan_rows(const uint16_t* h, const int32_t* sorted_ids, const int32_t* ntpp, int nslots,
+                                  int cols, int cap, unsigned* amax_bits, cudaStream_t stream);
+cudaError_t launch_quantize_tiles(const uint16_t* src, bool gather_x, const int32_t* sorted_ids, const int32_t* counts,
+                                  const int32_t* offsets, int E, int top_k, int nslots, int cols, int tiles_ub,
+                                  const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms, cudaStream_t stream);
+cudaError_t launch_nvfp4_up(const CUtensorMap& gate_codes, const CUtensorMap& up_codes, const CUtensorMap& x_codes,
+                            const Nvfp4GemmArgs& args, int num_sms, cudaStream_t stream);
+cudaError_t launch_nvfp4_down(const CUtensorMap& down_codes, const CUtensorMap& h_codes, const Nvfp4GemmArgs& args,
+                              int num_sms, cudaStream_t stream);
+
 }  // namespace moe

@@ -1,0 +1,173 @@
+"""GPU parity of the NVFP4 path (e2m1 weights and activations, e4m3 block-16 scales).
+
+* The GPU quantiser is bit-exact against the oracle's (codes, scales, global
+  scale): the same fp32 recipe takes every rounding decision on both sides.
+* The prepared blob keeps the codes and regroups the scales into 512-byte
+  atoms (checked against the atom index formula).
+* Grouped projections and the whole layer against the oracle's NVFP4 layer:
+  h elementwise as for bf16 (both sides quantise x identically, only the
+  accumulation order differs); y and out within the NVFP4 bound of
+  6e-2 x RMS (h is re-quantised from slightly different bf16 values).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import prefill_sigmoid_top_b200 as moe
+from prefill_sigmoid_top_b200 import inputs
+from tests._util import bf16_bits, bits_to_f64, rms
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def unpack_codes(packed):
+    p = np.asarray(packed, np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def _special_matrices():
+    rng = np.random.default_rng(3)
+    mats = []
+    m = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    m[0, :16] = 0.0                           # an all-zero block
+    m[1, :16] = 1e-30                         # a block far below the matrix amax
+    m[2, 16:32] = np.linspace(-3, 3, 16)      # includes exact e2m1 midpoints after scaling
+    mats.append(m)
+    mats.append((rng.standard_normal((64, 256)) * 50).astype(np.float32))
+    mats.append(np.zeros((64, 256), np.float32))  # amax 0 -> gs 1
+    return torch.tensor(np.stack(mats)).to(torch.bfloat16)
+
+
+def test_quantize_bitexact_against_oracle():
+    w = _special_matrices()
+    codes, scales, gs = moe.quantize_nvfp4(w.to(DEV))
+    torch.cuda.synchronize()
+    codes, scales, gs = unpack_codes(codes.cpu().numpy()), scales.cpu().numpy(), gs.cpu().numpy()
+    wb = bf16_bits(w)
+    for m in range(w.shape[0]):
+        oc, osc, ogs = oracle.nvfp4_quantize_bf16(wb[m])
+        assert np.float32(ogs) == gs[m]
+        assert np.array_equal(osc, scales[m])
+        assert np.array_equal(oc, codes[m])
+
+
+def test_quantize_bitexact_expert_weights():
+    cfg = inputs.CONFIGS[0].with_(E=4, I=256, H=512, seed=17)
+    wg, _, wd = inputs.expert_weights(cfg, DEV)
+    for w in (wg, wd):
+        codes, scales, gs = moe.quantize_nvfp4(w)
+        torch.cuda.synchronize()
+        codes, scales, gs = unpack_codes(codes.cpu().numpy()), scales.cpu().numpy(), gs.cpu().numpy()
+        for e in range(cfg.E):
+            oc, osc, ogs = oracle.nvfp4_quantize_bf16(bf16_bits(w[e]))
+            assert np.float32(ogs) == gs[e] and np.array_equal(osc, scales[e]) and np.array_equal(oc, codes[e])
+
+
+def test_prepared_blob_layout():
+    shape = moe.Shape(M=4, H=512, I=256, E=2, top_k=1, block_size=16)
+    w = torch.randn(2, 256, 512, device=DEV).to(torch.bfloat16)
+    codes, scales, gs = moe.quantize_nvfp4(w)
+    blob = moe.prepare_nvfp4_weights(codes, scales, shape, 0).cpu().numpy()
+    codes, scales = codes.cpu().numpy().reshape(512, 256), scales.cpu().numpy().reshape(512, 32)
+    nb = codes.size
+    assert np.array_equal(blob[:nb], codes.ravel())
+    atoms = blob[nb:]
+    assert atoms.size == scales.size
+    r, j = np.meshgrid(np.arange(512), np.arange(32), indexing="ij")
+    idx = ((r // 128) * 8 + j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4
+    assert np.array_equal(atoms[idx], scales)
+
+
+def _oracle_weights(d, E):
+    q = lambda t: [oracle.nvfp4_quantize_bf16(bf16_bits(t[e])) for e in range(E)]
+    return q(d["w_gate"]), q(d["w_up"]), q(d["w_down"])
+
+
+def _close(got, ref, rel, abs_rms):
+    tol = rel * np.abs(ref) + abs_rms * rms(ref)
+    d = np.abs(got - ref)
+    return (d <= tol).all(), float(d.max()), int((d > tol).sum())
+
+
+NVFP4_CASES = [dict(M=40, H=512, I=256, E=16, K=4, B=16), dict(M=300, H=256, I=512, E=8, K=4, B=16),
+               dict(M=7, H=768, I=256, E=32, K=6, B=32)]
+
+
+@pytest.mark.parametrize("case", NVFP4_CASES, ids=lambda c: f"M{c['M']}_E{c['E']}")
+def test_nvfp4_grouped_and_layer(case):
+    cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + 5, **case)
+    d = inputs.make_inputs(cfg, DEV)
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    nw = moe.nvfp4_weights(d["w_gate"], d["w_up"], d["w_down"], shape)
+    gq, uq, dq = _oracle_weights(d, cfg.E)
+    hb = dict(x=bf16_bits(d["x"]), wr=bf16_bits(d["w_router"]), b=d["bias"].cpu().numpy(), g=bf16_bits(d["gamma"]))
+    r = oracle.layer_nvfp4(hb["x"], hb["wr"], hb["b"], gq, uq, dq, hb["g"], cfg.eps, cfg.K)
+    # grouped projections on the oracle's plan
+    plan_o = oracle.align(r["ids_all"], cfg.E, cfg.B)
+    cap = moe.align_capacity(shape)
+    sorted_full = np.full(cap, -1, np.int32)
+    sorted_full[: plan_o["ntpp"]] = plan_o["sorted_ids"]
+    bexp = np.zeros(cap // cfg.B + 1, np.int32)
+    bexp[: len(plan_o["block_expert"])] = plan_o["block_expert"]
+    plan = dict(sorted_ids=torch.from_numpy(sorted_full).to(DEV), block_expert=torch.from_numpy(bexp).to(DEV),
+                expert_counts=torch.from_numpy(plan_o["counts"]).to(DEV),
+                expert_offsets=torch.from_numpy(plan_o["offsets"]).to(DEV),
+                num_tokens_post_padded=torch.tensor([plan_o["ntpp"]], dtype=torch.int32, device=DEV))
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    h = moe.grouped_up_swiglu_nvfp4(d["x"], nw, plan, shape, err_flag=err)
+    y = moe.grouped_down_nvfp4(h, nw, plan, shape, err_flag=err)
+    torch.cuda.synchronize()
+    assert moe.get_device_error(err) == 0
+    real = plan_o["sorted_ids"] < cfg.M * cfg.K
+    rows, slots = np.nonzero(real)[0], plan_o["sorted_ids"][real]
+    ok, e, nbad = _close(bits_to_f64(bf16_bits(h))[rows], bits_to_f64(r["h_all"])[slots], 2.0 ** -7, 1e-2)
+    assert ok, ("h", e, nbad)
+    y_ref = bits_to_f64(r["y"].reshape(cfg.M * cfg.K, cfg.H))
+    ok, e, nbad = _close(bits_to_f64(bf16_bits(y)), y_ref, 2.0 ** -3, 6e-2)
+    assert ok, ("y", e, nbad)
+    # the whole layer
+    ids = torch.empty(cfg.M, cfg.K, dtype=torch.int32, device=DEV)
+    out = moe.layer_nvfp4(d["x"], d["w_router"], d["bias"], nw, d["gamma"], cfg.eps, cfg.K, cfg.B, cfg.I,
+                          topk_ids=ids)
+    torch.cuda.synchronize()
+    assert np.array_equal(ids.cpu().numpy(), r["ids_all"])
+    ref = r["out_f64"]
+    assert np.abs(bits_to_f64(bf16_bits(out)) - ref).max() <= 6e-2 * rms(ref)
+
+
+def test_nvfp4_rejects_unsupported_intermediate():
+    shape = moe.Shape(M=4, H=256, I=128, E=2, top_k=1, block_size=16)  # I % 256 != 0
+    x = torch.zeros(4, 256, dtype=torch.bfloat16, device=DEV)
+    blob = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
+    gs = torch.ones(2, dtype=torch.float32, device=DEV)
+    nw = moe.NVFP4Weights(blob, blob, blob, gs, gs, gs)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.layer_nvfp4(x, torch.zeros(2, 256, dtype=torch.bfloat16, device=DEV), None, nw,
+                        torch.ones(256, dtype=torch.bfloat16, device=DEV), 1e-5, 1, 16, 128)
+    assert ei.value.status == 2
+
+
+@pytest.mark.slow
+def test_nvfp4_layer_full_size_sampled():
+    cfg = inputs.CONFIGS[4]
+    d = inputs.make_inputs(cfg, DEV)
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    nw = moe.nvfp4_weights(d["w_gate"], d["w_up"], d["w_down"], shape)
+    ids = torch.empty(cfg.M, cfg.K, dtype=torch.int32, device=DEV)
+    out = moe.layer_nvfp4(d["x"], d["w_router"], d["bias"], nw, d["gamma"], cfg.eps, cfg.K, cfg.B, cfg.I,
+                          topk_ids=ids)
+    torch.cuda.synchronize()
+    gq, uq, dq = _oracle_weights(d, cfg.E)
+    del d["w_gate"], d["w_up"], d["w_down"]
+    hb = dict(x=bf16_bits(d["x"]), wr=bf16_bits(d["w_router"]), b=d["bias"].cpu().numpy(), g=bf16_bits(d["gamma"]))
+    tokens = np.array([0, 1, 499, 998, 999], np.int32)
+    r = oracle.layer_nvfp4(hb["x"], hb["wr"], hb["b"], gq, uq, dq, hb["g"], cfg.eps, cfg.K, tokens=tokens)
+    assert np.array_equal(ids.cpu().numpy(), r["ids_all"])
+    ref = r["out_f64"]
+    got = bits_to_f64(bf16_bits(out))[tokens]
+    assert np.abs(got - ref).max() <= 6e-2 * rms(ref)
