@@ -9,9 +9,7 @@
 // (ascending slot id), so the plan is a deterministic function of topk_ids:
 //
 //  A. each warp owns one contiguous segment of the M*K slots and counts it
-//     into its own row of a [32][E] shared histogram (warp match_any gives
-//     the lanes holding the same expert; the group leader adds the group
-//     size, so no atomics are needed);
+//     into its own row of a [32][E] shared histogram;
 //  B. thread e sums its column -> expert_counts[e]; a block-wide exclusive
 //     scan of the padded counts -> prefix[]; barrier (the page's fix); then
 //     each column is turned into per-warp write cursors;
@@ -27,16 +25,21 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+// Dynamic shared memory budget: the 227 KB per-block limit minus room for the
+// kernel's static shared variables.
+constexpr size_t kSmemLimit = 227 * 1024 - 1024;
 
 __global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restrict__ topk_ids, int n, int E, int B,
                                                          int32_t* __restrict__ sorted_ids,
                                                          int32_t* __restrict__ block_expert,
                                                          int32_t* __restrict__ counts_out,
                                                          int32_t* __restrict__ offsets_out,
-                                                         int32_t* __restrict__ ntpp_out, int32_t* err) {
+                                                         int32_t* __restrict__ ntpp_out, int32_t* err,
+                                                         int stage_ids) {
   extern __shared__ int smem[];
   int* hist = smem;                  // [kWarps][E]: counts, then write cursors
   int* prefix = hist + kWarps * E;   // [E + 1]
+  int* staged = prefix + E + 1;      // [n] when stage_ids (they fit in shared memory)
   __shared__ int warp_sums[kWarps];
   __shared__ int bad;
 
@@ -45,21 +48,28 @@ __global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restri
 
   for (int i = tid; i < kWarps * E; i += kThreads) hist[i] = 0;
   if (tid == 0) bad = 0;
+  // Stage the ids once with all threads (many loads in flight), so the two
+  // in-order passes below read shared memory instead of waiting on global loads.
+  const bool use_staged = stage_ids != 0;
+  if (use_staged)
+    for (int i = tid; i < n; i += kThreads) staged[i] = topk_ids[i];
+  const int32_t* ids = use_staged ? staged : topk_ids;
   __syncthreads();
 
   const int seg = (n + kWarps - 1) / kWarps;
   const int f_begin = min(n, warp * seg), f_end = min(n, f_begin + seg);
 
-  // A: per-warp histogram of the segment
+  // A: per-warp histogram of the segment (shared-memory atomics: only the
+  // counts matter here, not the order)
   for (int base = f_begin; base < f_end; base += 32) {
     const int f = base + lane;
-    const bool act = f < f_end;
-    const int e = act ? topk_ids[f] : -1;
-    const bool ok = act && e >= 0 && e < E;
-    if (act && !ok) bad = 1;
-    const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1) & okmask;
-    if (ok && (__ffs(peers) - 1) == lane) hist[warp * E + e] += __popc(peers);
+    if (f < f_end) {
+      const int e = ids[f];
+      if (e >= 0 && e < E)
+        atomicAdd(&hist[warp * E + e], 1);
+      else
+        bad = 1;
+    }
   }
   __syncthreads();
   if (bad) {
@@ -117,7 +127,7 @@ __global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restri
   for (int base = f_begin; base < f_end; base += 32) {
     const int f = base + lane;
     const bool act = f < f_end;
-    const int e = act ? topk_ids[f] : -1;
+    const int e = act ? ids[f] : -1;
     const unsigned actmask = __ballot_sync(0xffffffffu, act);
     const unsigned peers = __match_any_sync(0xffffffffu, e) & actmask;
     int pos = 0;
@@ -152,16 +162,22 @@ __global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restri
 cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, int32_t* sorted_ids,
                          int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets, int32_t* ntpp,
                          int32_t* err, cudaStream_t stream) {
-  const size_t smem = sizeof(int) * (static_cast<size_t>(kWarps) * E + E + 1);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t st = cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(sizeof(int) * (kWarps * 1024 + 1025)));
+  const long long n = static_cast<long long>(M) * K;
+  const size_t base = sizeof(int) * (static_cast<size_t>(kWarps) * E + E + 1);
+  const bool stage = base + sizeof(int) * static_cast<size_t>(n) <= kSmemLimit;
+  const size_t smem = base + (stage ? sizeof(int) * static_cast<size_t>(n) : 0);
+  if (smem > kSmemLimit) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    st = cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
     if (st != cudaSuccess) return st;
-    attr_set = true;
+    attr_set[dev] = true;
   }
   align_kernel<<<1, kThreads, smem, stream>>>(topk_ids, M * K, E, B, sorted_ids, block_expert, expert_counts,
-                                             expert_offsets, ntpp, err);
+                                             expert_offsets, ntpp, err, stage ? 1 : 0);
   return cudaGetLastError();
 }
 

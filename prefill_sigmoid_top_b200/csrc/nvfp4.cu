@@ -211,9 +211,13 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(
   const int row0 = offsets[e] + local * 128;
   const float gs = nvfp4_global_scale(__uint_as_float(*amax_bits));
   const int nblk = cols / 16;
-  for (int idx = tid; idx < 128 * nblk; idx += blockDim.x) {
-    const int r = idx / nblk;
-    const int j = idx - r * nblk;
+  // this CTA's slice of 16-element column blocks: [jb0, jb1)
+  const int per = (nblk + gridDim.y - 1) / gridDim.y;
+  const int jb0 = blockIdx.y * per, jb1 = min(nblk, jb0 + per);
+  const int width = jb1 - jb0;
+  for (int idx = tid; idx < 128 * width; idx += blockDim.x) {
+    const int r = idx / width;
+    const int j = jb0 + (idx - r * width);
     uint32_t packed[2] = {0u, 0u};
     uint8_t sc = 0;
     if (r < nrows) {
@@ -595,8 +599,9 @@ cudaError_t launch_amax_plan_rows(const uint16_t* h, const int32_t* sorted_ids, 
 cudaError_t launch_quantize_tiles(const uint16_t* src, bool gather_x, const int32_t* sorted_ids, const int32_t* counts,
                                   const int32_t* offsets, int E, int top_k, int nslots, int cols, int tiles_ub,
                                   const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms, cudaStream_t stream) {
-  quantize_tiles_kernel<<<tiles_ub, 256, 0, stream>>>(src, gather_x, sorted_ids, counts, offsets, E, top_k, nslots,
-                                                      cols, amax_bits, codes, atoms);
+  const int slices = std::max(1, cols / 16 / 64);  // 64 column blocks (1024 elements) per CTA
+  quantize_tiles_kernel<<<dim3(tiles_ub, slices), 256, 0, stream>>>(src, gather_x, sorted_ids, counts, offsets, E,
+                                                                    top_k, nslots, cols, amax_bits, codes, atoms);
   return cudaGetLastError();
 }
 

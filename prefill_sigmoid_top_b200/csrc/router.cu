@@ -11,8 +11,9 @@
 //     lane partials are then combined with an xor butterfly (offsets 16, 8, 4,
 //     2, 1), which adds partial l and l+16 first, then the results 8 apart,
 //     and so on; the bias is added last.
-//     Register tiling: each lane carries 8 tokens x 4 experts partials, so a
-//     chunk of x and of w_router is loaded once per 32 fmas.
+//     Register tiling: each lane carries 8 tokens x 4 experts partials (1
+//     expert for small batches), so a chunk of x and of w_router is loaded
+//     once per 32 fmas; the next chunk is loaded while this one is used.
 //  2. router_topk_kernel: one warp per token selects the K largest logits
 //     (descending; equal logits -> lower expert id) by K rounds of a warp
 //     argmax, then w_k = s_k / sum s with s = 1 / (1 + exp(-z)).
@@ -25,7 +26,6 @@ namespace moe {
 namespace {
 
 constexpr int kTokPerWarp = 8;
-constexpr int kExpPerWarp = 4;
 constexpr int kWarps = 4;
 
 __device__ __forceinline__ uint4 ld_nc_16(const uint16_t* p) {
@@ -41,55 +41,75 @@ __device__ __forceinline__ float elem(const uint4& v, int i) {
   return (i & 1) ? bf16_hi(w) : bf16_lo(w);
 }
 
+// kExp experts x 8 tokens of partials per lane.  With kPipe the next chunk's
+// loads are issued before the current chunk's fmas (software pipelining), so
+// the L2 latency of one chunk hides behind the arithmetic of the previous one;
+// it doubles the load registers, so it is used where there are few warps.
+template <int kExp, bool kPipe>
 __global__ void __launch_bounds__(kWarps * 32) router_logits_kernel(const uint16_t* __restrict__ x,
                                                                     const uint16_t* __restrict__ w_router,
                                                                     const float* __restrict__ bias, int M, int H,
                                                                     int E, float* __restrict__ logits) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kTokPerWarp;
-  const int e0 = (blockIdx.y * kWarps + warp) * kExpPerWarp;
+  const int e0 = (blockIdx.y * kWarps + warp) * kExp;
   if (e0 >= E) return;
 
-  float acc[kTokPerWarp][kExpPerWarp];
+  float acc[kTokPerWarp][kExp];
 #pragma unroll
   for (int t = 0; t < kTokPerWarp; ++t)
 #pragma unroll
-    for (int q = 0; q < kExpPerWarp; ++q) acc[t][q] = 0.0f;
+    for (int q = 0; q < kExp; ++q) acc[t][q] = 0.0f;
 
   const int nchunk = H / 256;
-#pragma unroll 1
-  for (int j = 0; j < nchunk; ++j) {
+  uint4 wv[kExp], xv[kTokPerWarp];
+  auto load = [&](int j, uint4 (&wd)[kExp], uint4 (&xd)[kTokPerWarp]) {
     const int h = 256 * j + 8 * lane;
-    uint4 wv[kExpPerWarp], xv[kTokPerWarp];
 #pragma unroll
-    for (int q = 0; q < kExpPerWarp; ++q)
-      wv[q] = (e0 + q < E) ? ld_nc_16(w_router + static_cast<size_t>(e0 + q) * H + h) : make_uint4(0, 0, 0, 0);
+    for (int q = 0; q < kExp; ++q)
+      wd[q] = (e0 + q < E) ? ld_nc_16(w_router + static_cast<size_t>(e0 + q) * H + h) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int t = 0; t < kTokPerWarp; ++t)
-      xv[t] = (t0 + t < M) ? ld_nc_16(x + static_cast<size_t>(t0 + t) * H + h) : make_uint4(0, 0, 0, 0);
+      xd[t] = (t0 + t < M) ? ld_nc_16(x + static_cast<size_t>(t0 + t) * H + h) : make_uint4(0, 0, 0, 0);
+  };
+  if (kPipe) load(0, wv, xv);
+#pragma unroll 1
+  for (int j = 0; j < nchunk; ++j) {
+    uint4 wn[kExp], xn[kTokPerWarp];
+    if (kPipe) {
+      if (j + 1 < nchunk) load(j + 1, wn, xn);
+    } else {
+      load(j, wv, xv);
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i)  // increasing h inside the chunk
 #pragma unroll
       for (int t = 0; t < kTokPerWarp; ++t)
 #pragma unroll
-        for (int q = 0; q < kExpPerWarp; ++q) acc[t][q] = __fmaf_rn(elem(xv[t], i), elem(wv[q], i), acc[t][q]);
+        for (int q = 0; q < kExp; ++q) acc[t][q] = __fmaf_rn(elem(xv[t], i), elem(wv[q], i), acc[t][q]);
+    if (kPipe && j + 1 < nchunk) {
+#pragma unroll
+      for (int q = 0; q < kExp; ++q) wv[q] = wn[q];
+#pragma unroll
+      for (int t = 0; t < kTokPerWarp; ++t) xv[t] = xn[t];
+    }
   }
 
 #pragma unroll
   for (int t = 0; t < kTokPerWarp; ++t)
 #pragma unroll
-    for (int q = 0; q < kExpPerWarp; ++q) {
+    for (int q = 0; q < kExp; ++q) {
       float v = acc[t][q];
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
       acc[t][q] = v;
     }
-  // lane l stores pair l = (t, q) = (l / 4, l % 4)
+  // lane l stores pair l = (t, q) = (l / kExp, l % kExp)
 #pragma unroll
   for (int t = 0; t < kTokPerWarp; ++t)
 #pragma unroll
-    for (int q = 0; q < kExpPerWarp; ++q)
-      if (lane == t * kExpPerWarp + q && t0 + t < M && e0 + q < E) {
+    for (int q = 0; q < kExp; ++q)
+      if (lane == t * kExp + q && t0 + t < M && e0 + q < E) {
         const float b = bias != nullptr ? bias[e0 + q] : 0.0f;
         logits[static_cast<size_t>(t0 + t) * E + e0 + q] = __fadd_rn(acc[t][q], b);
       }
@@ -157,9 +177,14 @@ __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restric
 
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
                                  float* logits, cudaStream_t stream) {
-  const int experts_per_block = kWarps * kExpPerWarp;
-  dim3 grid((M + kTokPerWarp - 1) / kTokPerWarp, (E + experts_per_block - 1) / experts_per_block);
-  router_logits_kernel<<<grid, kWarps * 32, 0, stream>>>(x, w_router, bias, M, H, E, logits);
+  const int tok_blocks = (M + kTokPerWarp - 1) / kTokPerWarp;
+  if (M <= 64) {  // few tokens: one expert per warp, so that enough warps stream W_r
+    dim3 grid(tok_blocks, (E + kWarps - 1) / kWarps);
+    router_logits_kernel<1, true><<<grid, kWarps * 32, 0, stream>>>(x, w_router, bias, M, H, E, logits);
+  } else {
+    dim3 grid(tok_blocks, (E + 4 * kWarps - 1) / (4 * kWarps));
+    router_logits_kernel<4, false><<<grid, kWarps * 32, 0, stream>>>(x, w_router, bias, M, H, E, logits);
+  }
   return cudaGetLastError();
 }
 
