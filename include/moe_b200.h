@@ -256,6 +256,12 @@ MOE_API moe_status_t moe_route_noalloc(const moe_bf16_t* x, const moe_bf16_t* w_
  * *host_code, MOE_OK or the most severe device-detected status
  * (MOE_ERR_TIMEOUT before MOE_ERR_INVALID_INPUT).  Clears nothing. */
 MOE_API moe_status_t moe_get_device_error(const int32_t* err_flag, moe_stream_t stream, int32_t* host_code);
+
+/* Failure-path self-test: launches one warp whose bounded wait (the same wait
+ * the pipelined kernels use on their mbarriers) can never be satisfied; after
+ * limit_us (1 .. 1,000,000) it ORs the MOE_ERR_TIMEOUT bit into *err_flag and
+ * returns.  Nothing faults, traps or hangs; the stream stays usable. */
+MOE_API moe_status_t moe_selftest_wait_timeout(int32_t* err_flag, uint32_t limit_us, moe_stream_t stream);
 MOE_API const char* moe_status_string(moe_status_t status);
 
 #ifdef __cplusplus

@@ -102,6 +102,7 @@ def _declare(L):
         "moe_nvfp4_blob_bytes": (sz, [_Shape, ctypes.c_int]),
         "moe_get_device_error": (st, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
         "moe_route_noalloc": (st, [vp, vp, vp, _Shape, vp, vp, vp]),
+        "moe_selftest_wait_timeout": (st, [vp, ctypes.c_uint32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -388,6 +389,11 @@ def layer_nvfp4(x, w_router, bias, nw: NVFP4Weights, gamma, eps, top_k, block_si
                                _ptr(_bf16(gamma)), float(eps), shape.c(), _ptr(out), _ptr(residual_out),
                                _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_layer")
     return out
+
+
+def selftest_wait_timeout(err_flag, limit_us: int = 1000):
+    """Run the kernel whose bounded wait always expires (see moe_selftest_wait_timeout)."""
+    _check(library().moe_selftest_wait_timeout(_ptr(err_flag), int(limit_us), _stream()), "moe_selftest_wait_timeout")
 
 
 def get_device_error(err_flag) -> int:

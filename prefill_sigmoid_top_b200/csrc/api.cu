@@ -598,6 +598,13 @@ size_t moe_nvfp4_blob_bytes(moe_shape_t s, int which) {
   return static_cast<size_t>(rows) * cols / 2 + static_cast<size_t>(rows) * cols / 16;
 }
 
+moe_status_t moe_selftest_wait_timeout(int32_t* err_flag, uint32_t limit_us, moe_stream_t stream) {
+  if (!err_flag) return MOE_ERR_INVALID_ARG;
+  if (limit_us == 0 || limit_us > 1000000u) return MOE_ERR_INVALID_ARG;
+  return cuda_status(moe::launch_wait_timeout_selftest(err_flag, static_cast<uint64_t>(limit_us) * 1000ull,
+                                                       static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_get_device_error(const int32_t* err_flag, moe_stream_t stream, int32_t* host_code) {
   if (!err_flag || !host_code) return MOE_ERR_INVALID_ARG;
   int32_t v = 0;

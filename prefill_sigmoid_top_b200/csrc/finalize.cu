@@ -4,18 +4,20 @@
 // token, 7 vectors of bf16x8 per thread = 896 packs = one H=7168 row; §3:
 // RMS_EPS = 1e-5 and WEIGHT_BIAS = 0, so gamma multiplies as is).
 //
-// One CTA of 128 threads per token.  Each thread owns up to 8 packs of 8
-// hidden elements (p = tid + 128*i), keeps s = x + sum_k w_k * y_k for them
-// in 64 fp32 registers, and only out (and optionally bf16(s)) is written:
-// the expert sum never goes back to HBM before the norm.
+// One CTA of 256 threads per token.  Each thread owns up to 4 packs of 8
+// hidden elements (p = tid + 256*i), keeps s = x + sum_k w_k * y_k for them
+// in 32 fp32 registers, and only out (and optionally bf16(s)) is written:
+// the expert sum never goes back to HBM before the norm.  The loop over the
+// K expert rows is unrolled by 4, so 16 independent 16-byte loads per thread
+// are in flight.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kMaxPacks = 8;  // H <= 8 * 8 * 128 = 8192
+constexpr int kThreads = 256;
+constexpr int kMaxPacks = 4;  // H <= 4 * 8 * 256 = 8192
 
 __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
   uint4 v;
@@ -54,7 +56,7 @@ __global__ void __launch_bounds__(kThreads) finalize_kernel(const uint16_t* __re
     }
   }
   const uint16_t* yt = y + static_cast<size_t>(t) * K * H;
-#pragma unroll 2
+#pragma unroll 4
   for (int k = 0; k < K; ++k) {
     const float wk = topk_w[static_cast<size_t>(t) * K + k];
     uint4 v[kMaxPacks];
@@ -109,7 +111,25 @@ __global__ void __launch_bounds__(kThreads) finalize_kernel(const uint16_t* __re
   }
 }
 
+// Self-test of the bounded waits every pipelined kernel uses: thread 0 waits
+// on an mbarrier that nothing ever arrives at, gives up after limit_ns and
+// records MOE_ERR_TIMEOUT, exactly as a kernel whose copies never landed would.
+__global__ void wait_timeout_selftest_kernel(int32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, nullptr, limit_ns)) set_error(err, kErrTimeout);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_selftest(int32_t* err, uint64_t limit_ns, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(err, limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_finalize(const uint16_t* x, const uint16_t* y, const float* topk_w, const uint16_t* gamma,
                             float eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out,

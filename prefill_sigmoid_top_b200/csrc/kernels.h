@@ -30,6 +30,9 @@ cudaError_t launch_finalize(const uint16_t* x, const uint16_t* y, const float* t
                             float eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out,
                             cudaStream_t stream);
 
+// finalize.cu: one-warp kernel whose bounded wait can never be satisfied.
+cudaError_t launch_wait_timeout_selftest(int32_t* err, uint64_t limit_ns, cudaStream_t stream);
+
 // gemm_bf16.cu: grouped projections over the expert-major plan.
 struct GroupedGemmArgs {
   const int32_t* sorted_ids;

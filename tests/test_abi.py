@@ -106,3 +106,10 @@ def test_layer_workspace_checks():
 def test_device_error_rejects_null():
     code = ctypes.c_int32(0)
     assert moe.library().moe_get_device_error(None, None, ctypes.byref(code)) == 1
+
+
+def test_selftest_rejects_bad_arguments():
+    L = moe.library()
+    assert L.moe_selftest_wait_timeout(None, 1000, None) == 1
+    assert L.moe_selftest_wait_timeout(FAKE, 0, None) == 1
+    assert L.moe_selftest_wait_timeout(FAKE, 2_000_000, None) == 1

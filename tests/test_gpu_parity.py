@@ -389,3 +389,12 @@ def test_layer_cuda_graph_replay():
         torch.cuda.synchronize()
         assert torch.equal(out, eager)
     del graph
+
+
+# ------------------------------------------------------------------ failure path
+def test_bounded_wait_times_out_and_device_stays_usable():
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.selftest_wait_timeout(err, limit_us=2000)
+    assert moe.get_device_error(err) == 5  # MOE_ERR_TIMEOUT, reported on the host
+    # the context is intact: a layer runs and matches the oracle afterwards
+    test_layer_small(LAYER_SMALL[0])
