@@ -7,7 +7,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/moe_b200.h"
+#include "moe_b200.h"
 #include "common.cuh"
 #include "kernels.h"
 

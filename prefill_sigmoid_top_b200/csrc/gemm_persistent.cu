@@ -172,30 +172,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ weight producer
+    // lane 0 waits for the slot and posts the byte count; lanes 0 and 1 then
+    // issue one box each, so the two copies of a stage are issued in parallel.
     if (lane == 0) {
       prefetch_tensor_map(&tm_a0);
       if (kUp) prefetch_tensor_map(&tm_a1);
-      int ka = 0;
-      bool alive = true;
-      for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
-        const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
-        const bool single_use = cnt[c.e] <= kNmax;
-        const uint64_t pol = single_use ? l2_policy_evict_first() : l2_policy_evict_normal();
-        const int row_a0 = kUp ? c.e * args.rows_per_expert + c.w * kBM : c.e * args.rows_per_expert + c.w * 2 * kBM;
-        const int row_a1 = kUp ? row_a0 : row_a0 + kBM;
-        for (int k = 0; k < nk; ++k, ++ka) {
-          const int s = ka % kStagesA;
-          if (!mbar_wait_bounded(&a_empty[s], ((ka / kStagesA) & 1) ^ 1, abort_flag)) {
+    }
+    int ka = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
+      const bool single_use = cnt[c.e] <= kNmax;
+      const uint64_t pol = single_use ? l2_policy_evict_first() : l2_policy_evict_normal();
+      const int row_a0 = kUp ? c.e * args.rows_per_expert + c.w * kBM : c.e * args.rows_per_expert + c.w * 2 * kBM;
+      const int row_a1 = kUp ? row_a0 : row_a0 + kBM;
+      for (int k = 0; k < nk; ++k, ++ka) {
+        const int s = ka % kStagesA;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&a_empty[s], ((ka / kStagesA) & 1) ^ 1, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&a_full[s], C::kAStage);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
             *abort_flag = 1;
             set_error(args.err, kErrTimeout);
-            alive = false;
-            break;
           }
-          uint8_t* st = a_ring + s * C::kAStage;
-          mbar_arrive_expect_tx(&a_full[s], C::kAStage);
-          tma_load_2d_hint(&tm_a0, &a_full[s], st, k * kBK, row_a0, pol);
-          tma_load_2d_hint(kUp ? &tm_a1 : &tm_a0, &a_full[s], st + kBoxBytes, k * kBK, row_a1, pol);
+          alive = false;
+          break;
         }
+        uint8_t* st = a_ring + s * C::kAStage;
+        if (lane == 0)
+          tma_load_2d_hint(&tm_a0, &a_full[s], st, k * kBK, row_a0, pol);
+        else if (lane == 1)
+          tma_load_2d_hint(kUp ? &tm_a1 : &tm_a0, &a_full[s], st + kBoxBytes, k * kBK, row_a1, pol);
       }
     }
     __syncwarp();
@@ -252,28 +263,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------ token-row producer (plan-ordered rows)
-    if (lane == 0) {
-      prefetch_tensor_map(&tm_b);
-      int kb = 0;
-      bool alive = true;
-      for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
-        const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
-        const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
-        const int row0 = args.expert_offsets[c.e] + c.t * kNmax;
-        const int nbox = (nrows + kBRows - 1) / kBRows;
-        for (int k = 0; k < nk; ++k, ++kb) {
-          const int s = kb % kStagesB;
-          if (!mbar_wait_bounded(&b_empty[s], ((kb / kStagesB) & 1) ^ 1, abort_flag)) {
+    // lane 0 waits and posts the byte count; lane i issues box i.
+    if (lane == 0) prefetch_tensor_map(&tm_b);
+    int kb = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
+      const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
+      const int row0 = args.expert_offsets[c.e] + c.t * kNmax;
+      const int nbox = (nrows + kBRows - 1) / kBRows;
+      for (int k = 0; k < nk; ++k, ++kb) {
+        const int s = kb % kStagesB;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&b_empty[s], ((kb / kStagesB) & 1) ^ 1, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&b_full[s], nbox * kBRows * kBK * 2);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
             *abort_flag = 1;
             set_error(args.err, kErrTimeout);
-            alive = false;
-            break;
           }
-          uint8_t* st = b_ring + s * C::kBStage;
-          mbar_arrive_expect_tx(&b_full[s], nbox * kBRows * kBK * 2);
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(&tm_b, &b_full[s], st + i * kBRows * kBK * 2, k * kBK, row0 + i * kBRows);
+          alive = false;
+          break;
         }
+        uint8_t* st = b_ring + s * C::kBStage;
+        if (lane < nbox)
+          tma_load_2d(&tm_b, &b_full[s], st + lane * kBRows * kBK * 2, k * kBK, row0 + lane * kBRows);
       }
     }
     __syncwarp();

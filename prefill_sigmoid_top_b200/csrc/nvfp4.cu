@@ -350,59 +350,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ weight producer (codes + scales)
-    if (lane == 0) {
-      int ka = 0;
-      bool alive = true;
-      for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
-        const TileCoord c = decode_tile(prefix, cnt, E, tile);
-        const uint64_t pol = cnt[c.e] <= kNmax ? l2_policy_evict_first() : l2_policy_evict_normal();
-        const int row_a0 = kUp ? c.e * g.rows_per_expert + c.w * kBM : c.e * g.rows_per_expert + c.w * 2 * kBM;
-        const int row_a1 = kUp ? row_a0 : row_a0 + kBM;
-        const uint8_t* sf0 = args.sfa0 + static_cast<int64_t>(row_a0 / kBM) * kblk64 * 512;
-        const uint8_t* sf1 = args.sfa1 + static_cast<int64_t>(row_a1 / kBM) * kblk64 * 512;
-        for (int k = 0; k < nk; ++k, ++ka) {
-          const int s = ka % kStagesA;
-          if (!mbar_wait_bounded(&a_empty[s], ((ka / kStagesA) & 1) ^ 1, abort_flag)) {
+    // lane 0 waits for the slot and posts the byte count; lanes 0-3 issue the
+    // stage's two code boxes and two scale copies in parallel.
+    int ka = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
+      const TileCoord c = decode_tile(prefix, cnt, E, tile);
+      const uint64_t pol = cnt[c.e] <= kNmax ? l2_policy_evict_first() : l2_policy_evict_normal();
+      const int row_a0 = kUp ? c.e * g.rows_per_expert + c.w * kBM : c.e * g.rows_per_expert + c.w * 2 * kBM;
+      const int row_a1 = kUp ? row_a0 : row_a0 + kBM;
+      const uint8_t* sf0 = args.sfa0 + static_cast<int64_t>(row_a0 / kBM) * kblk64 * 512;
+      const uint8_t* sf1 = args.sfa1 + static_cast<int64_t>(row_a1 / kBM) * kblk64 * 512;
+      for (int k = 0; k < nk; ++k, ++ka) {
+        const int s = ka % kStagesA;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&a_empty[s], ((ka / kStagesA) & 1) ^ 1, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&a_full[s], kAStage);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
             *abort_flag = 1;
             set_error(g.err, kErrTimeout);
-            alive = false;
-            break;
           }
-          uint8_t* st = a_ring + s * kAStage;
-          mbar_arrive_expect_tx(&a_full[s], kAStage);
-          tma_load_2d_hint(&tm_a0, &a_full[s], st, k * 128, row_a0, pol);
-          tma_load_2d_hint(kUp ? &tm_a1 : &tm_a0, &a_full[s], st + kBoxBytes, k * 128, row_a1, pol);
-          bulk_load(st + 2 * kBoxBytes, sf0 + k * kSfChunk, kSfChunk, &a_full[s]);
-          bulk_load(st + 2 * kBoxBytes + kSfChunk, sf1 + k * kSfChunk, kSfChunk, &a_full[s]);
+          alive = false;
+          break;
         }
+        uint8_t* st = a_ring + s * kAStage;
+        if (lane == 0)
+          tma_load_2d_hint(&tm_a0, &a_full[s], st, k * 128, row_a0, pol);
+        else if (lane == 1)
+          tma_load_2d_hint(kUp ? &tm_a1 : &tm_a0, &a_full[s], st + kBoxBytes, k * 128, row_a1, pol);
+        else if (lane == 2)
+          bulk_load(st + 2 * kBoxBytes, sf0 + k * kSfChunk, kSfChunk, &a_full[s]);
+        else if (lane == 3)
+          bulk_load(st + 2 * kBoxBytes + kSfChunk, sf1 + k * kSfChunk, kSfChunk, &a_full[s]);
       }
     }
     __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------ activation producer (tile-aligned codes + scales)
-    if (lane == 0) {
-      int kb = 0;
-      bool alive = true;
-      for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
-        const TileCoord c = decode_tile(prefix, cnt, E, tile);
-        const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
-        const int ti = prefix[c.e] / W + c.t;  // global token-tile index
-        const int nbox = (nrows + kBRows - 1) / kBRows;
-        const uint8_t* sfb = args.sfb + static_cast<int64_t>(ti) * kblk64 * 512;
-        for (int k = 0; k < nk; ++k, ++kb) {
-          const int s = kb % kStagesB;
-          if (!mbar_wait_bounded(&b_empty[s], ((kb / kStagesB) & 1) ^ 1, abort_flag)) {
+    int kb = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
+      const TileCoord c = decode_tile(prefix, cnt, E, tile);
+      const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
+      const int ti = prefix[c.e] / W + c.t;  // global token-tile index
+      const int nbox = (nrows + kBRows - 1) / kBRows;
+      const uint8_t* sfb = args.sfb + static_cast<int64_t>(ti) * kblk64 * 512;
+      for (int k = 0; k < nk; ++k, ++kb) {
+        const int s = kb % kStagesB;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&b_empty[s], ((kb / kStagesB) & 1) ^ 1, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&b_full[s], nbox * kBRows * 128 + kSfChunk);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
             *abort_flag = 1;
             set_error(g.err, kErrTimeout);
-            alive = false;
-            break;
           }
-          uint8_t* st = b_ring + s * kBStage;
-          mbar_arrive_expect_tx(&b_full[s], nbox * kBRows * 128 + kSfChunk);
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(&tm_b, &b_full[s], st + i * kBRows * 128, k * 128, ti * kNmax + i * kBRows);
-          bulk_load(st + kNmax * 128, sfb + k * kSfChunk, kSfChunk, &b_full[s]);
+          alive = false;
+          break;
         }
+        uint8_t* st = b_ring + s * kBStage;
+        if (lane < nbox)
+          tma_load_2d(&tm_b, &b_full[s], st + lane * kBRows * 128, k * 128, ti * kNmax + lane * kBRows);
+        else if (lane == 31)
+          bulk_load(st + kNmax * 128, sfb + k * kSfChunk, kSfChunk, &b_full[s]);
       }
     }
     __syncwarp();
