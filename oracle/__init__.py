@@ -55,6 +55,7 @@ def lib():
                 "oracle_e4m3_encode": (ctypes.c_uint8, [f32]),
                 "oracle_router_logits": (None, [vp, vp, vp, i32, i32, i32, vp, vp]),
                 "oracle_topk": (None, [vp, i32, i32, i32, vp, vp]),
+                "oracle_topk_ex": (None, [vp, i32, i32, i32, i32, i32, f64, vp, vp]),
                 "oracle_align": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
                 "oracle_expert": (None, [vp, vp, vp, vp, i32, i32, vp, vp]),
                 "oracle_finalize": (None, [vp, vp, vp, vp, f64, i32, i32, i32, vp, vp, vp, vp]),
@@ -145,6 +146,23 @@ def topk(z32, K):
 
 def route(x, w_router, bias, K):
     return topk(router_logits(x, w_router, bias), K)
+
+
+SCORING_SOFTMAX, SCORING_SIGMOID = 0, 1
+
+
+def topk_ex(z32, K, scoring=SCORING_SIGMOID, renormalize=True, scale=1.0):
+    """Selection as topk(); weights from sigmoid or softmax scores, optionally renormalised, times scale."""
+    z32 = np.ascontiguousarray(z32, dtype=np.float32)
+    M, E = z32.shape
+    ids = np.empty((M, K), np.int32)
+    w = np.empty((M, K), np.float64)
+    lib().oracle_topk_ex(_p(z32), M, E, K, int(scoring), int(bool(renormalize)), float(scale), _p(ids), _p(w))
+    return ids, w
+
+
+def route_ex(x, w_router, bias, K, scoring=SCORING_SIGMOID, renormalize=True, scale=1.0):
+    return topk_ex(router_logits(x, w_router, bias), K, scoring, renormalize, scale)
 
 
 # ------------------------------------------------------------------ align

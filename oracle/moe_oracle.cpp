@@ -250,6 +250,36 @@ void oracle_topk(const float* z32, int M, int E, int K, int32_t* topk_ids, doubl
   }
 }
 
+// Routing variants (sglang PR #29509 analysis, §2: the fused top-k takes a
+// norm_type, 0 = softmax scoring and 1 = sigmoid scoring).  Selection is the
+// same as oracle_topk (the K largest fp32 logits; both scores are monotone in
+// the logit).  Scores and weights in fp64:
+//   scoring 1 (sigmoid): p_k = sigmoid(z_k)
+//   scoring 0 (softmax): p_k = exp(z_k - zmax) / sum_e exp(z_e - zmax), over all E
+//   w_k = p_k / sum_j p_j if renormalize, else p_k; then w_k *= scale
+void oracle_topk_ex(const float* z32, int M, int E, int K, int scoring, int renormalize, double scale,
+                    int32_t* topk_ids, double* topk_w) {
+  std::vector<double> dummy(static_cast<size_t>(M) * K);
+  oracle_topk(z32, M, E, K, topk_ids, dummy.data());
+  for (int t = 0; t < M; ++t) {
+    const float* z = z32 + static_cast<size_t>(t) * E;
+    double p[64];
+    double denom_all = 0.0, zmax = -INFINITY;
+    if (scoring == 0) {
+      for (int e = 0; e < E; ++e) zmax = std::max(zmax, static_cast<double>(z[e]));
+      for (int e = 0; e < E; ++e) denom_all += std::exp(static_cast<double>(z[e]) - zmax);
+    }
+    double total = 0.0;
+    for (int k = 0; k < K; ++k) {
+      const double zk = static_cast<double>(z[topk_ids[static_cast<size_t>(t) * K + k]]);
+      p[k] = scoring == 0 ? std::exp(zk - zmax) / denom_all : sigmoid(zk);
+      total += p[k];
+    }
+    for (int k = 0; k < K; ++k)
+      topk_w[static_cast<size_t>(t) * K + k] = (renormalize ? p[k] / total : p[k]) * scale;
+  }
+}
+
 // ------------------------------------------------------------ align --------
 // Expert-major block plan (flashinfer PR #6511 analysis, §5): histogram of
 // the flat slots f = t*K + k by expert; padded exclusive prefix where each

@@ -125,3 +125,29 @@ def test_route_all_configs_shapes_small():
     # the canonical order needs H % 256 == 0; every workload satisfies it
     for cfg in inputs.CONFIGS.values():
         assert cfg.H % 256 == 0 and cfg.K <= cfg.E
+
+
+# ------------------------------------------------------------------ routing variants
+@pytest.mark.parametrize("renormalize", [True, False])
+@pytest.mark.parametrize("scale", [1.0, 2.5])
+def test_softmax_scoring_matches_scipy(renormalize, scale):
+    rng = np.random.default_rng(31)
+    z = (rng.standard_normal((40, 64)) * 3).astype(np.float32)
+    ids, w = oracle.topk_ex(z, 6, oracle.SCORING_SOFTMAX, renormalize, scale)
+    ids_s, _ = oracle.topk(z, 6)
+    assert np.array_equal(ids, ids_s)                 # selection is the same
+    p = scipy.special.softmax(z.astype(np.float64), axis=1)  # library softmax over all experts
+    sel = np.take_along_axis(p, ids, axis=1)
+    ref = (sel / sel.sum(axis=1, keepdims=True) if renormalize else sel) * scale
+    assert np.allclose(w, ref, rtol=1e-12, atol=0)
+
+
+def test_sigmoid_without_renormalisation_is_the_score():
+    rng = np.random.default_rng(32)
+    z = rng.standard_normal((20, 32)).astype(np.float32)
+    ids, w = oracle.topk_ex(z, 4, oracle.SCORING_SIGMOID, False, 1.0)
+    assert np.allclose(w, scipy.special.expit(np.take_along_axis(z, ids, axis=1).astype(np.float64)),
+                       rtol=1e-13, atol=0)
+    ids2, w2 = oracle.topk_ex(z, 4, oracle.SCORING_SIGMOID, True, 1.0)
+    ids3, w3 = oracle.topk(z, 4)
+    assert np.array_equal(ids2, ids3) and np.allclose(w2, w3, rtol=1e-15, atol=0)
