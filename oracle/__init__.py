@@ -55,7 +55,7 @@ def lib():
                 "oracle_e4m3_encode": (ctypes.c_uint8, [f32]),
                 "oracle_router_logits": (None, [vp, vp, vp, i32, i32, i32, vp, vp]),
                 "oracle_topk": (None, [vp, i32, i32, i32, vp, vp]),
-                "oracle_topk_ex": (None, [vp, i32, i32, i32, i32, i32, f64, vp, vp]),
+                "oracle_topk_ex": (None, [vp, vp, i32, i32, i32, i32, i32, f64, vp, vp]),
                 "oracle_align": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
                 "oracle_expert": (None, [vp, vp, vp, vp, i32, i32, vp, vp]),
                 "oracle_finalize": (None, [vp, vp, vp, vp, f64, i32, i32, i32, vp, vp, vp, vp]),
@@ -151,18 +151,25 @@ def route(x, w_router, bias, K):
 SCORING_SOFTMAX, SCORING_SIGMOID = 0, 1
 
 
-def topk_ex(z32, K, scoring=SCORING_SIGMOID, renormalize=True, scale=1.0):
-    """Selection as topk(); weights from sigmoid or softmax scores, optionally renormalised, times scale."""
+def topk_ex(z32, K, scoring=SCORING_SIGMOID, renormalize=True, scale=1.0, sel_bias=None):
+    """Selection on fp32(z32 + sel_bias) (sel_bias None -> on z32), as topk(); weights from the sigmoid
+    or softmax score of z32, optionally renormalised over the K selected, times scale."""
     z32 = np.ascontiguousarray(z32, dtype=np.float32)
     M, E = z32.shape
+    b = None if sel_bias is None else np.ascontiguousarray(sel_bias, dtype=np.float32)
     ids = np.empty((M, K), np.int32)
     w = np.empty((M, K), np.float64)
-    lib().oracle_topk_ex(_p(z32), M, E, K, int(scoring), int(bool(renormalize)), float(scale), _p(ids), _p(w))
+    lib().oracle_topk_ex(_p(z32), _p(b), M, E, K, int(scoring), int(bool(renormalize)), float(scale), _p(ids),
+                         _p(w))
     return ids, w
 
 
-def route_ex(x, w_router, bias, K, scoring=SCORING_SIGMOID, renormalize=True, scale=1.0):
-    return topk_ex(router_logits(x, w_router, bias), K, scoring, renormalize, scale)
+def route_ex(x, w_router, bias, K, scoring=SCORING_SIGMOID, renormalize=True, scale=1.0, bias_in_score=True):
+    """Routing variants.  bias_in_score: the bias is part of the logit (as route()); otherwise it only
+    shifts the selection key and the score is taken from the logit without it."""
+    if bias_in_score or bias is None:
+        return topk_ex(router_logits(x, w_router, bias), K, scoring, renormalize, scale)
+    return topk_ex(router_logits(x, w_router, None), K, scoring, renormalize, scale, sel_bias=bias)
 
 
 # ------------------------------------------------------------------ align

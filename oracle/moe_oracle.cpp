@@ -251,16 +251,24 @@ void oracle_topk(const float* z32, int M, int E, int K, int32_t* topk_ids, doubl
 }
 
 // Routing variants (sglang PR #29509 analysis, §2: the fused top-k takes a
-// norm_type, 0 = softmax scoring and 1 = sigmoid scoring).  Selection is the
-// same as oracle_topk (the K largest fp32 logits; both scores are monotone in
-// the logit).  Scores and weights in fp64:
+// norm_type, 0 = softmax scoring and 1 = sigmoid scoring).  z32 is the
+// canonical logit; sel_bias (nullable) is a per-expert bias that enters only
+// the selection key, key = fp32(z + sel_bias[e]), and not the score.  The K
+// experts are those oracle_topk picks on the key.  Scores and weights in fp64:
 //   scoring 1 (sigmoid): p_k = sigmoid(z_k)
 //   scoring 0 (softmax): p_k = exp(z_k - zmax) / sum_e exp(z_e - zmax), over all E
 //   w_k = p_k / sum_j p_j if renormalize, else p_k; then w_k *= scale
-void oracle_topk_ex(const float* z32, int M, int E, int K, int scoring, int renormalize, double scale,
-                    int32_t* topk_ids, double* topk_w) {
-  std::vector<double> dummy(static_cast<size_t>(M) * K);
-  oracle_topk(z32, M, E, K, topk_ids, dummy.data());
+void oracle_topk_ex(const float* z32, const float* sel_bias, int M, int E, int K, int scoring, int renormalize,
+                    double scale, int32_t* topk_ids, double* topk_w) {
+  std::vector<float> key(z32, z32 + static_cast<size_t>(M) * E);
+  if (sel_bias != nullptr)
+    for (int t = 0; t < M; ++t)
+      for (int e = 0; e < E; ++e) {
+        volatile float sum = key[static_cast<size_t>(t) * E + e] + sel_bias[e];  // one fp32 add
+        key[static_cast<size_t>(t) * E + e] = sum;
+      }
+  std::vector<double> unused(static_cast<size_t>(M) * K);
+  oracle_topk(key.data(), M, E, K, topk_ids, unused.data());
   for (int t = 0; t < M; ++t) {
     const float* z = z32 + static_cast<size_t>(t) * E;
     double p[64];

@@ -151,3 +151,20 @@ def test_sigmoid_without_renormalisation_is_the_score():
     ids2, w2 = oracle.topk_ex(z, 4, oracle.SCORING_SIGMOID, True, 1.0)
     ids3, w3 = oracle.topk(z, 4)
     assert np.array_equal(ids2, ids3) and np.allclose(w2, w3, rtol=1e-15, atol=0)
+
+
+def test_selection_only_bias():
+    # The bias shifts which experts are picked but not their weights: the picked set is the one the
+    # biased logit picks, and the weights are the renormalised sigmoid of the unbiased logit.
+    cfg = inputs.CONFIGS[0].with_(M=24, H=512, E=32, K=4)
+    w_router, bias, gamma, x = inputs.router_inputs(cfg)
+    b = (np.arange(cfg.E, dtype=np.float32) - cfg.E / 2) * 0.25   # large enough to change the picks
+    ids, w = oracle.route_ex(bf16_bits(x), bf16_bits(w_router), b, cfg.K, bias_in_score=False)
+    ids_biased, _ = oracle.route(bf16_bits(x), bf16_bits(w_router), b, cfg.K)
+    assert np.array_equal(ids, ids_biased)
+    z = oracle.router_logits(bf16_bits(x), bf16_bits(w_router), None).astype(np.float64)
+    s = scipy.special.expit(np.take_along_axis(z, ids, axis=1))
+    assert np.allclose(w, s / s.sum(axis=1, keepdims=True), rtol=1e-13, atol=0)
+    # and the picks differ from the unbiased ones somewhere, so the bias did act
+    ids_plain, _ = oracle.route(bf16_bits(x), bf16_bits(w_router), None, cfg.K)
+    assert not np.array_equal(ids, ids_plain)
