@@ -119,6 +119,31 @@ MOE_API moe_status_t moe_route(const moe_bf16_t* x, const moe_bf16_t* w_router, 
                        int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream);
 MOE_API size_t moe_route_workspace_size(moe_shape_t s);
 
+/* -------------------------------------------------------- route variants --
+ * The routing variants of the same fused top-k (sglang PR #29509 analysis,
+ * §2: its norm_type selects softmax (0) or sigmoid (1) scores).
+ * The selection key is z as above, except that with bias_in_score == 0 the
+ * bias is left out of z and added to the key only: key = fp32(z + bias[e]).
+ * topk_ids = the K largest keys, descending, ties -> lower id.  With z_k the
+ * logit (bias_in_score == 0: without the bias) of the k-th selected expert:
+ *   scoring SIGMOID: p_k = 1 / (1 + exp(-z_k))
+ *   scoring SOFTMAX: p_k = exp(z_k) / sum_e exp(z[t,e]), over all E experts
+ *   w_k = (renormalize ? p_k / sum_j p_j : p_k) * routed_scale
+ * {SIGMOID, renormalize 1, bias_in_score 1, routed_scale 1} is moe_route.
+ * Arguments, layouts, workspace and errors as moe_route; opts is a host
+ * pointer, read during the call; INVALID_ARG for a null opts, an unknown
+ * scoring, or a routed_scale that is not finite and > 0. */
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
+typedef struct {
+  int32_t scoring;       /* moe_score_t */
+  int32_t renormalize;   /* nonzero: renormalise over the K selected */
+  int32_t bias_in_score; /* nonzero: bias is part of z; zero: it shifts the selection key only */
+  float routed_scale;    /* multiplies every weight */
+} moe_route_opts_t;
+MOE_API moe_status_t moe_route_ex(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, moe_shape_t s,
+                                  const moe_route_opts_t* opts, int32_t* topk_ids, float* topk_w, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- align --
  * Expert-major block plan (flashinfer PR #6511 analysis, §5).
  *   expert_counts[e]      = #{f : topk_ids[f] == e}, f = t*K + k

@@ -56,6 +56,13 @@ class _Plan(ctypes.Structure):
                 ("num_tokens_post_padded", ctypes.c_void_p)]
 
 
+class _RouteOpts(ctypes.Structure):
+    _fields_ = [("scoring", ctypes.c_int32), ("renormalize", ctypes.c_int32), ("bias_in_score", ctypes.c_int32),
+                ("routed_scale", ctypes.c_float)]
+
+
+SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
+
 _LAYOUT_FIELDS = ["err_flag", "logits", "topk_ids", "topk_w", "sorted_ids", "block_expert", "expert_counts",
                   "expert_offsets", "num_tokens_post_padded", "h", "y", "act_scratch", "total"]
 
@@ -83,6 +90,7 @@ def _declare(L):
         "moe_status_string": (ctypes.c_char_p, [st]),
         "moe_route": (st, [vp, vp, vp, _Shape, vp, vp, vp, sz, vp]),
         "moe_route_workspace_size": (sz, [_Shape]),
+        "moe_route_ex": (st, [vp, vp, vp, _Shape, ctypes.POINTER(_RouteOpts), vp, vp, vp, sz, vp]),
         "moe_align_block_size": (st, [vp, _Shape, vp, vp, vp, vp, vp, vp, vp]),
         "moe_align_capacity": (sz, [_Shape]),
         "moe_grouped_up_swiglu": (st, [vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Plan), _Shape, vp, vp, sz,
@@ -192,6 +200,27 @@ def route(x, w_router, bias, top_k, topk_ids=None, topk_w=None, ws=None):
         ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     _check(library().moe_route(_ptr(_bf16(x)), _ptr(_bf16(w_router)), _ptr(bias), shape.c(), _ptr(topk_ids),
                                _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_route")
+    return topk_ids, topk_w
+
+
+def route_ex(x, w_router, bias, top_k, scoring=SCORE_SIGMOID, renormalize=True, routed_scale=1.0,
+             bias_in_score=True, topk_ids=None, topk_w=None, ws=None):
+    """Routing variants: softmax or sigmoid scores, optional renormalisation, a routed scale, and a bias
+    that is part of the logit or only shifts the selection key -> (topk_ids, topk_w)."""
+    _need_cuda(x, w_router, bias)
+    M, H = x.shape
+    E = w_router.shape[0]
+    shape = Shape(M, H, 128, E, top_k, 16)
+    if topk_ids is None:
+        topk_ids = torch.empty(M, top_k, dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty(M, top_k, dtype=torch.float32, device=x.device)
+    need = route_workspace_size(shape)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    opts = _RouteOpts(int(scoring), int(bool(renormalize)), int(bool(bias_in_score)), float(routed_scale))
+    _check(library().moe_route_ex(_ptr(_bf16(x)), _ptr(_bf16(w_router)), _ptr(bias), shape.c(), ctypes.byref(opts),
+                                  _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream()), "moe_route_ex")
     return topk_ids, topk_w
 
 

@@ -3,6 +3,7 @@
 // workspace layout, and the launch sequence of the layer.
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -440,6 +441,26 @@ moe_status_t moe_route(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs));
   if (st != MOE_OK) return st;
   return cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, topk_ids, topk_w, cs));
+}
+
+moe_status_t moe_route_ex(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, moe_shape_t s,
+                          const moe_route_opts_t* opts, int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!x || !w_router || !topk_ids || !topk_w || !opts) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+  if (opts->scoring != MOE_SCORE_SOFTMAX && opts->scoring != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (!(opts->routed_scale > 0.0f) || !std::isfinite(opts->routed_scale)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_route_workspace_size(s)) return MOE_ERR_WORKSPACE;
+  auto cs = static_cast<cudaStream_t>(stream);
+  float* logits = static_cast<float*>(ws);
+  const bool sel_only = bias != nullptr && opts->bias_in_score == 0;
+  st = cuda_status(moe::launch_router_logits(x, w_router, sel_only ? nullptr : bias, s.M, s.H, s.E, logits, cs));
+  if (st != MOE_OK) return st;
+  return cuda_status(moe::launch_router_topk_ext(logits, sel_only ? bias : nullptr, s.M, s.E, s.top_k, opts->scoring,
+                                                 opts->renormalize != 0 ? 1 : 0, opts->routed_scale, topk_ids,
+                                                 topk_w, cs));
 }
 
 moe_status_t moe_align_block_size(const int32_t* topk_ids, moe_shape_t s, int32_t* sorted_ids, int32_t* block_expert,

@@ -19,6 +19,9 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, co
                                  float* logits, cudaStream_t stream);
 cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t* topk_ids, float* topk_w,
                                cudaStream_t stream);
+cudaError_t launch_router_topk_ext(const float* logits, const float* sel_bias, int M, int E, int K, int scoring,
+                                   int renormalize, float scale, int32_t* topk_ids, float* topk_w,
+                                   cudaStream_t stream);
 
 // align.cu
 cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, int32_t* sorted_ids,

@@ -17,6 +17,11 @@
 //  2. router_topk_kernel: one warp per token selects the K largest logits
 //     (descending; equal logits -> lower expert id) by K rounds of a warp
 //     argmax, then w_k = s_k / sum s with s = 1 / (1 + exp(-z)).
+//  2'. router_topk_ext_kernel: the routing variants of the same page (its
+//     norm_type: 0 = softmax, 1 = sigmoid scores), optional renormalisation,
+//     a routed scale, and a bias that only shifts the selection key.  The
+//     selection is the same warp argmax on the key; the score of a selected
+//     expert is taken from the logit without the selection-only bias.
 #include <mutex>
 
 #include "common.cuh"
@@ -173,6 +178,79 @@ __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restric
   }
 }
 
+template <int kPerLane>
+__global__ void __launch_bounds__(128) router_topk_ext_kernel(const float* __restrict__ logits,
+                                                              const float* __restrict__ sel_bias, int M, int E,
+                                                              int K, int scoring, int renormalize, float scale,
+                                                              int32_t* __restrict__ topk_ids,
+                                                              float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (t >= M) return;
+  const float* zt = logits + static_cast<size_t>(t) * E;
+  float z[kPerLane], v[kPerLane];
+  bool live[kPerLane];
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int e = lane + 32 * i;
+    live[i] = e < E;
+    z[i] = live[i] ? zt[e] : -INFINITY;
+    v[i] = (live[i] && sel_bias != nullptr) ? __fadd_rn(z[i], sel_bias[e]) : z[i];
+  }
+  // softmax over all E experts: max, then the sum of exp(z - max)
+  float zmax = -INFINITY, denom = 0.0f;
+  if (scoring == MOE_SCORE_SOFTMAX) {
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) zmax = fmaxf(zmax, z[i]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, off));
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)
+      if (live[i]) denom += expf(z[i] - zmax);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, off);
+  }
+  int sel_id = 0;
+  for (int k = 0; k < K; ++k) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)
+      if (live[i] && better(v[i], lane + 32 * i, bv, bi)) {
+        bv = v[i];
+        bi = lane + 32 * i;
+      }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i)
+      if (lane + 32 * i == bi) live[i] = false;
+    if (lane == k) sel_id = bi;
+  }
+  float p = 0.0f;
+  if (lane < K) {
+    const float zs = zt[sel_id];
+    if (scoring == MOE_SCORE_SOFTMAX)  // the common 1/denom cancels when renormalising
+      p = renormalize ? expf(zs - zmax) : expf(zs - zmax) / denom;
+    else
+      p = 1.0f / (1.0f + expf(-zs));
+  }
+  float total = p;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+  if (lane < K) {
+    topk_ids[static_cast<size_t>(t) * K + lane] = sel_id;
+    topk_w[static_cast<size_t>(t) * K + lane] = (renormalize ? p / total : p) * scale;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
@@ -197,6 +275,22 @@ cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t
     router_topk_kernel<8><<<grid, 128, 0, stream>>>(logits, M, E, K, topk_ids, topk_w);
   else
     router_topk_kernel<32><<<grid, 128, 0, stream>>>(logits, M, E, K, topk_ids, topk_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_topk_ext(const float* logits, const float* sel_bias, int M, int E, int K, int scoring,
+                                   int renormalize, float scale, int32_t* topk_ids, float* topk_w,
+                                   cudaStream_t stream) {
+  dim3 grid((M + 3) / 4);
+  if (E <= 64)
+    router_topk_ext_kernel<2><<<grid, 128, 0, stream>>>(logits, sel_bias, M, E, K, scoring, renormalize, scale,
+                                                        topk_ids, topk_w);
+  else if (E <= 256)
+    router_topk_ext_kernel<8><<<grid, 128, 0, stream>>>(logits, sel_bias, M, E, K, scoring, renormalize, scale,
+                                                        topk_ids, topk_w);
+  else
+    router_topk_ext_kernel<32><<<grid, 128, 0, stream>>>(logits, sel_bias, M, E, K, scoring, renormalize, scale,
+                                                         topk_ids, topk_w);
   return cudaGetLastError();
 }
 

@@ -10,7 +10,7 @@ import re
 import pytest
 
 import prefill_sigmoid_top_b200 as moe
-from prefill_sigmoid_top_b200 import _Plan, _Shape, _Weights, _Layout
+from prefill_sigmoid_top_b200 import _Plan, _Shape, _Weights, _Layout, _RouteOpts
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe_b200.h")
@@ -113,3 +113,17 @@ def test_selftest_rejects_bad_arguments():
     assert L.moe_selftest_wait_timeout(None, 1000, None) == 1
     assert L.moe_selftest_wait_timeout(FAKE, 0, None) == 1
     assert L.moe_selftest_wait_timeout(FAKE, 2_000_000, None) == 1
+
+
+def test_route_ex_rejects_bad_options():
+    L = moe.library()
+    s = C0.c()
+    ok = _RouteOpts(moe.SCORE_SOFTMAX, 1, 1, 1.0)
+    args = lambda o: (FAKE, FAKE, None, s, o, FAKE, FAKE, FAKE, 1 << 20, None)
+    assert L.moe_route_ex(*args(None)) == 1
+    assert L.moe_route_ex(*args(ctypes.byref(_RouteOpts(2, 1, 1, 1.0)))) == 1
+    assert L.moe_route_ex(*args(ctypes.byref(_RouteOpts(1, 1, 1, 0.0)))) == 1
+    assert L.moe_route_ex(*args(ctypes.byref(_RouteOpts(1, 1, 1, float("inf"))))) == 1
+    assert L.moe_route_ex(*args(ctypes.byref(_RouteOpts(1, 1, 1, float("nan"))))) == 1
+    assert L.moe_route_ex(FAKE, FAKE, None, s, ctypes.byref(ok), FAKE, FAKE, FAKE, 4, None) == 3
+    assert L.moe_route_ex(FAKE_MIS, FAKE, None, s, ctypes.byref(ok), FAKE, FAKE, FAKE, 1 << 20, None) == 1
