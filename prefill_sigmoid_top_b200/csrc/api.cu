@@ -124,19 +124,25 @@ int nvfp4_tiles_ub(const moe_shape_t& s) {
   const long long mk = static_cast<long long>(s.M) * s.top_k;
   return static_cast<int>(mk / 128 + (mk < s.E ? mk : s.E));
 }
-// Tile-aligned NVFP4 activation copy of `cols`-wide rows: amax word, codes, scale atoms.
+// Tile-aligned NVFP4 activation copy of `cols`-wide rows: amax word, codes,
+// scale atoms; for x (per_token) also the per-token codes and scales it is
+// gathered from.
 struct ActLayout {
-  size_t amax, codes, atoms, total;
+  size_t amax, codes, atoms, tok_codes, tok_scales, total;
 };
-ActLayout act_layout(const moe_shape_t& s, int cols) {
+ActLayout act_layout(const moe_shape_t& s, int cols, bool per_token) {
   ActLayout L{};
   const size_t rows = static_cast<size_t>(nvfp4_tiles_ub(s)) * 128;
   L.amax = 0;
   L.codes = kAlign;
   L.atoms = align_up(L.codes + rows * cols / 2);
-  L.total = align_up(L.atoms + static_cast<size_t>(nvfp4_tiles_ub(s)) * (cols / 64) * 512);
+  L.tok_codes = align_up(L.atoms + static_cast<size_t>(nvfp4_tiles_ub(s)) * (cols / 64) * 512);
+  L.tok_scales = per_token ? align_up(L.tok_codes + static_cast<size_t>(s.M) * cols / 2) : L.tok_codes;
+  L.total = per_token ? align_up(L.tok_scales + static_cast<size_t>(s.M) * cols / 16) : L.tok_codes;
   return L;
 }
+ActLayout x_act_layout(const moe_shape_t& s) { return act_layout(s, s.H, true); }
+ActLayout h_act_layout(const moe_shape_t& s) { return act_layout(s, s.I, false); }
 // Blob of one projection: codes [rows, cols/2] then scale atoms.
 void blob_dims(const moe_shape_t& s, int which, int64_t* rows, int64_t* cols) {
   *rows = static_cast<int64_t>(s.E) * (which == 2 ? s.H : s.I);
@@ -271,14 +277,17 @@ int num_sms();
 
 moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
                           const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream) {
-  const ActLayout L = act_layout(s, s.H);
+  const ActLayout L = x_act_layout(s);
   auto* base = static_cast<uint8_t*>(ws);
   auto* amax = reinterpret_cast<unsigned*>(base + L.amax);
   const int tiles = nvfp4_tiles_ub(s);
   if (cudaMemsetAsync(amax, 0, sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
   if (moe::launch_amax_all(x, static_cast<int64_t>(s.M) * s.H, amax, stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (moe::launch_quantize_tiles(x, true, plan->sorted_ids, plan->expert_counts, plan->expert_offsets, s.E, s.top_k,
-                                 s.M * s.top_k, s.H, tiles, amax, base + L.codes, base + L.atoms, stream) != cudaSuccess)
+  if (moe::launch_quantize_rows(x, s.M, s.H, amax, base + L.tok_codes, base + L.tok_scales, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::launch_gather_tiles(base + L.tok_codes, base + L.tok_scales, plan->sorted_ids, plan->expert_counts,
+                               plan->expert_offsets, s.E, s.top_k, s.M * s.top_k, s.H, tiles, base + L.codes,
+                               base + L.atoms, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   CUtensorMap mg, mu, mx;
   const uint64_t wrows = static_cast<uint64_t>(s.E) * s.I;
@@ -308,7 +317,7 @@ moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe
 
 moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
                             const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream) {
-  const ActLayout L = act_layout(s, s.I);
+  const ActLayout L = h_act_layout(s);
   auto* base = static_cast<uint8_t*>(ws);
   auto* amax = reinterpret_cast<unsigned*>(base + L.amax);
   const int tiles = nvfp4_tiles_ub(s);
@@ -316,8 +325,8 @@ moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const m
   if (moe::launch_amax_plan_rows(h, plan->sorted_ids, plan->num_tokens_post_padded, s.M * s.top_k, s.I,
                                  static_cast<int>(cap_rows(s)), amax, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (moe::launch_quantize_tiles(h, false, plan->sorted_ids, plan->expert_counts, plan->expert_offsets, s.E, s.top_k,
-                                 s.M * s.top_k, s.I, tiles, amax, base + L.codes, base + L.atoms, stream) != cudaSuccess)
+  if (moe::launch_quantize_tiles(h, plan->expert_counts, plan->expert_offsets, s.E, s.I, tiles, amax, base + L.codes,
+                                 base + L.atoms, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   CUtensorMap md, mh;
   if (!make_map_u8(&md, w->down, static_cast<uint64_t>(s.E) * s.H, s.I / 2, 128) ||
@@ -373,7 +382,7 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   off = align_up(off + mk * s.H * sizeof(uint16_t));
   L.act_scratch = off;  // bf16: x gathered into plan order; NVFP4: the two tile-aligned activation copies
   if (dt == MOE_W_NVFP4)
-    off = align_up(off + act_layout(s, s.H).total + act_layout(s, s.I).total);
+    off = align_up(off + x_act_layout(s).total + h_act_layout(s).total);
   else
     off = align_up(off + pregather_bytes(s));
   L.total = off;
@@ -420,13 +429,13 @@ size_t moe_route_workspace_size(moe_shape_t s) {
 
 size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK) return 0;
-  if (dtype == MOE_W_NVFP4) return act_layout(s, s.H).total;
+  if (dtype == MOE_W_NVFP4) return x_act_layout(s).total;
   return (want_pregather(s) || want_persistent(s)) ? pregather_bytes(s) : 0;
 }
 
 size_t moe_down_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK) return 0;
-  return dtype == MOE_W_NVFP4 ? act_layout(s, s.I).total : 0;
+  return dtype == MOE_W_NVFP4 ? h_act_layout(s).total : 0;
 }
 
 moe_status_t moe_route(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, moe_shape_t s,
@@ -574,7 +583,7 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   if (w->dtype == MOE_W_NVFP4) {
     uint8_t* act = base + L.act_scratch;
     if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs)) != MOE_OK) return st;
-    if ((st = run_down_nvfp4(h, w, &plan, s, y, act + act_layout(s, s.H).total, err, cs)) != MOE_OK) return st;
+    if ((st = run_down_nvfp4(h, w, &plan, s, y, act + x_act_layout(s).total, err, cs)) != MOE_OK) return st;
   } else {
     if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
     if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;

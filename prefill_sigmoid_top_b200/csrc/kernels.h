@@ -95,9 +95,17 @@ cudaError_t launch_nvfp4_scales_to_atoms(const uint8_t* scales, int64_t rows, in
 cudaError_t launch_amax_all(const uint16_t* src, int64_t n, unsigned* amax_bits, cudaStream_t stream);
 cudaError_t launch_amax_plan_rows(const uint16_t* h, const int32_t* sorted_ids, const int32_t* ntpp, int nslots,
                                   int cols, int cap, unsigned* amax_bits, cudaStream_t stream);
-cudaError_t launch_quantize_tiles(const uint16_t* src, bool gather_x, const int32_t* sorted_ids, const int32_t* counts,
-                                  const int32_t* offsets, int E, int top_k, int nslots, int cols, int tiles_ub,
-                                  const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms, cudaStream_t stream);
+// h (plan order) -> tile-aligned NVFP4 codes / scale atoms (global scale from *amax_bits).
+cudaError_t launch_quantize_tiles(const uint16_t* src, const int32_t* counts, const int32_t* offsets, int E, int cols,
+                                  int tiles_ub, const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms,
+                                  cudaStream_t stream);
+// rows x cols bf16 -> codes [rows, cols/2], row-major scales [rows, cols/16] (global scale from *amax_bits).
+cudaError_t launch_quantize_rows(const uint16_t* src, int64_t rows, int64_t cols, const unsigned* amax_bits,
+                                 uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+// per-token codes / scales -> tile-aligned copy of the routed slots (row r of tile ti <- token sorted_ids[..] / top_k).
+cudaError_t launch_gather_tiles(const uint8_t* tok_codes, const uint8_t* tok_scales, const int32_t* sorted_ids,
+                                const int32_t* counts, const int32_t* offsets, int E, int top_k, int nslots, int cols,
+                                int tiles_ub, uint8_t* codes, uint8_t* atoms, cudaStream_t stream);
 cudaError_t launch_nvfp4_up(const CUtensorMap& gate_codes, const CUtensorMap& up_codes, const CUtensorMap& x_codes,
                             const Nvfp4GemmArgs& args, int num_sms, cudaStream_t stream);
 cudaError_t launch_nvfp4_down(const CUtensorMap& down_codes, const CUtensorMap& h_codes, const Nvfp4GemmArgs& args,

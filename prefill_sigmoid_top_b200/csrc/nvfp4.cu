@@ -164,21 +164,13 @@ __global__ void __launch_bounds__(256) plan_rows_amax_kernel(const uint16_t* __r
   block_max_to(amax_bits, mx);
 }
 
-// Token tile `blockIdx.x` (global numbering: expert by expert, ceil(count/128)
-// tiles each) -> rows [128 ti, 128 ti + 128) of the tile-aligned NVFP4 copy.
-// gather_x: the source rows are x[sorted_ids[r] / top_k]; else h[r] (plan order).
-// Padding rows (beyond the expert's count) are written as zero codes / scales.
-__global__ void __launch_bounds__(256) quantize_tiles_kernel(
-    const uint16_t* __restrict__ src, bool gather_x, const int32_t* __restrict__ sorted_ids,
-    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int E, int top_k, int nslots, int cols,
-    const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ atoms) {
-  __shared__ int s_cnt[1024];
-  __shared__ int s_info[2];
+// Which expert owns token tile ti (tiles numbered expert by expert,
+// ceil(count/128) each): after the call s_info = {expert or -1, tile index
+// inside the expert}.  Every thread calls it; s_cnt holds the counts.
+__device__ void locate_tile(const int* s_cnt, int E, int ti, int* s_info) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = counts[e];
   if (tid == 0) s_info[0] = -1;
   __syncthreads();
-  const int ti = blockIdx.x;
   if (warp == 0) {
     const int per = (E + 31) / 32;
     const int lo = min(E, lane * per), hi = min(E, lo + per);
@@ -204,6 +196,23 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(
     }
   }
   __syncthreads();
+}
+
+// Token tile `blockIdx.x` -> rows [128 ti, 128 ti + nrows) of the tile-aligned
+// NVFP4 copy of h (plan order, `cols` wide): codes and scale atoms.  Rows past
+// the expert's count are not written: the GEMM computes their columns from
+// whatever they hold and never stores them (a column of the product depends
+// on its own row of this operand only).
+__global__ void __launch_bounds__(256) quantize_tiles_kernel(
+    const uint16_t* __restrict__ src, const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int E,
+    int cols, const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ atoms) {
+  __shared__ int s_cnt[1024];
+  __shared__ int s_info[2];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = counts[e];
+  __syncthreads();
+  const int ti = blockIdx.x;
+  locate_tile(s_cnt, E, ti, s_info);
   const int e = s_info[0];
   if (e < 0) return;
   const int local = s_info[1];
@@ -215,26 +224,55 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(
   const int per = (nblk + gridDim.y - 1) / gridDim.y;
   const int jb0 = blockIdx.y * per, jb1 = min(nblk, jb0 + per);
   const int width = jb1 - jb0;
-  for (int idx = tid; idx < 128 * width; idx += blockDim.x) {
+  for (int idx = tid; idx < nrows * width; idx += blockDim.x) {
     const int r = idx / width;
     const int j = jb0 + (idx - r * width);
-    uint32_t packed[2] = {0u, 0u};
-    uint8_t sc = 0;
-    if (r < nrows) {
-      const uint16_t* row;
-      if (gather_x) {
-        const int id = sorted_ids[row0 + r];
-        row = src + static_cast<int64_t>((id >= 0 && id < nslots) ? id / top_k : 0) * cols;
-      } else {
-        row = src + static_cast<int64_t>(row0 + r) * cols;
-      }
-      float v[16];
-      load16_bf16(row + j * 16, v);
-      sc = quantize_block16(v, gs, packed);
-    }
+    float v[16];
+    load16_bf16(src + static_cast<int64_t>(row0 + r) * cols + j * 16, v);
+    uint32_t packed[2];
+    const uint8_t sc = quantize_block16(v, gs, packed);
     *reinterpret_cast<uint2*>(codes + (static_cast<int64_t>(ti) * 128 + r) * (cols / 2) + j * 8) =
         make_uint2(packed[0], packed[1]);
     atoms[(static_cast<int64_t>(ti) * (cols / 64) + j / 4) * 512 + (r % 32) * 16 + (r / 32) * 4 + (j % 4)] = sc;
+  }
+}
+
+// x enters the up projection once per routed slot, i.e. up to top_k times per
+// token, so it is quantised once per token (quantize_kernel) and this kernel
+// copies each slot's codes and scales into the tile-aligned layout: token tile
+// `blockIdx.x`, row r <- token sorted_ids[row0 + r] / top_k.  One warp per row;
+// a row's scales (cols/16 bytes) move as 4-byte words, each word the four
+// column blocks of one scale atom row.  Rows past the expert's count are not
+// written (as above).
+__global__ void __launch_bounds__(256) gather_tiles_kernel(
+    const uint8_t* __restrict__ tok_codes, const uint8_t* __restrict__ tok_scales,
+    const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+    int E, int top_k, int nslots, int cols, uint8_t* __restrict__ codes, uint8_t* __restrict__ atoms) {
+  __shared__ int s_cnt[1024];
+  __shared__ int s_info[2];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = counts[e];
+  __syncthreads();
+  const int ti = blockIdx.x;
+  locate_tile(s_cnt, E, ti, s_info);
+  const int e = s_info[0];
+  if (e < 0) return;
+  const int local = s_info[1];
+  const int nrows = min(128, s_cnt[e] - local * 128);
+  const int row0 = offsets[e] + local * 128;
+  const int cb16 = cols / 32;  // 16-byte code chunks per row
+  const int nw = cols / 64;    // scale words per row
+  for (int r = warp; r < nrows; r += blockDim.x / 32) {
+    const int id = sorted_ids[row0 + r];
+    const int t = (id >= 0 && id < nslots) ? id / top_k : -1;
+    const uint4* src = reinterpret_cast<const uint4*>(tok_codes + static_cast<int64_t>(t < 0 ? 0 : t) * (cols / 2));
+    uint4* dst = reinterpret_cast<uint4*>(codes + (static_cast<int64_t>(ti) * 128 + r) * (cols / 2));
+    for (int c = lane; c < cb16; c += 32) dst[c] = t >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
+    const uint32_t* ssrc =
+        reinterpret_cast<const uint32_t*>(tok_scales + static_cast<int64_t>(t < 0 ? 0 : t) * (cols / 16));
+    for (int a = lane; a < nw; a += 32)
+      *reinterpret_cast<uint32_t*>(atoms + (static_cast<int64_t>(ti) * nw + a) * 512 + (r % 32) * 16 + (r / 32) * 4) =
+          t >= 0 ? ssrc[a] : 0u;
   }
 }
 
@@ -613,12 +651,29 @@ cudaError_t launch_amax_plan_rows(const uint16_t* h, const int32_t* sorted_ids, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_tiles(const uint16_t* src, bool gather_x, const int32_t* sorted_ids, const int32_t* counts,
-                                  const int32_t* offsets, int E, int top_k, int nslots, int cols, int tiles_ub,
-                                  const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms, cudaStream_t stream) {
+cudaError_t launch_quantize_tiles(const uint16_t* src, const int32_t* counts, const int32_t* offsets, int E, int cols,
+                                  int tiles_ub, const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms,
+                                  cudaStream_t stream) {
   const int slices = std::max(1, cols / 16 / 64);  // 64 column blocks (1024 elements) per CTA
-  quantize_tiles_kernel<<<dim3(tiles_ub, slices), 256, 0, stream>>>(src, gather_x, sorted_ids, counts, offsets, E,
-                                                                    top_k, nslots, cols, amax_bits, codes, atoms);
+  quantize_tiles_kernel<<<dim3(tiles_ub, slices), 256, 0, stream>>>(src, counts, offsets, E, cols, amax_bits, codes,
+                                                                    atoms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(const uint16_t* src, int64_t rows, int64_t cols, const unsigned* amax_bits,
+                                 uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
+  const int64_t total_blocks = rows * (cols / 16);
+  const int64_t grid = std::min<int64_t>((total_blocks + 255) / 256, 148 * 16);
+  quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(src, total_blocks, cols / 16, rows, amax_bits,
+                                                                   codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_tiles(const uint8_t* tok_codes, const uint8_t* tok_scales, const int32_t* sorted_ids,
+                                const int32_t* counts, const int32_t* offsets, int E, int top_k, int nslots, int cols,
+                                int tiles_ub, uint8_t* codes, uint8_t* atoms, cudaStream_t stream) {
+  gather_tiles_kernel<<<tiles_ub, 256, 0, stream>>>(tok_codes, tok_scales, sorted_ids, counts, offsets, E, top_k,
+                                                    nslots, cols, codes, atoms);
   return cudaGetLastError();
 }
 

@@ -3,17 +3,18 @@
 // norm_type=1, rather than softmax).
 //
 // Two launches:
-//  1. router_logits_kernel: z[t,e] = x[t] . w_router[e] + bias[e] in fp32, in
-//     the canonical order that makes the selection reproducible bit for bit:
-//     lane l of a warp accumulates, one fma per element and in increasing h,
-//     the elements h = 256*j + 8*l + i (i = 0..7, j = 0..H/256-1), i.e. the
-//     16-byte chunk the lane loads in a coalesced 512-byte warp load; the 32
-//     lane partials are then combined with an xor butterfly (offsets 16, 8, 4,
-//     2, 1), which adds partial l and l+16 first, then the results 8 apart,
-//     and so on; the bias is added last.
-//     Register tiling: each lane carries 8 tokens x 4 experts partials (1
-//     expert for small batches), so a chunk of x and of w_router is loaded
-//     once per 32 fmas; the next chunk is loaded while this one is used.
+//  1. router_logits_staged_kernel: z[t,e] = x[t] . w_router[e] + bias[e] in
+//     fp32, in the canonical order that makes the selection reproducible bit
+//     for bit: partial l (l = 0..31) accumulates, one fma per element and in
+//     increasing h, the elements h = 256*j + 8*l + i (i = 0..7, j = 0..H/256-1);
+//     the 32 partials are then combined with an xor butterfly (offsets 16, 8,
+//     4, 2, 1), which adds partial l and l+16 first, then the results 8
+//     apart, and so on; the bias is added last.  Lane l of a warp owns
+//     partial l of each of the warp's (token, expert) pairs; x and w_router
+//     arrive through a shared-memory ring of 256-element slabs (cp.async).
+//     Few tokens: 8 tokens x 1 expert per warp, 16 slabs in flight.  Many
+//     tokens: 8 tokens x 8 experts per warp, the fmas of token pairs issued
+//     as paired fp32 fmas.
 //  2. router_topk_kernel: one warp per token selects the K largest logits
 //     (descending; equal logits -> lower expert id) by K rounds of a warp
 //     argmax, then w_k = s_k / sum s with s = 1 / (1 + exp(-z)).
@@ -30,94 +31,192 @@
 namespace moe {
 namespace {
 
-constexpr int kTokPerWarp = 8;
-constexpr int kWarps = 4;
-
-__device__ __forceinline__ uint4 ld_nc_16(const uint16_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ float elem(const uint4& v, int i) {
   const uint32_t w = (i < 2) ? v.x : (i < 4) ? v.y : (i < 6) ? v.z : v.w;
   return (i & 1) ? bf16_hi(w) : bf16_lo(w);
 }
 
-// kExp experts x 8 tokens of partials per lane.  With kPipe the next chunk's
-// loads are issued before the current chunk's fmas (software pipelining), so
-// the L2 latency of one chunk hides behind the arithmetic of the previous one;
-// it doubles the load registers, so it is used where there are few warps.
-template <int kExp, bool kPipe>
-__global__ void __launch_bounds__(kWarps * 32) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                                    const uint16_t* __restrict__ w_router,
-                                                                    const float* __restrict__ bias, int M, int H,
-                                                                    int E, float* __restrict__ logits) {
+// ---------------------------------------------------------------------------
+// Logits.  x and w_router reach the warps through a ring of kStages slabs of
+// 256 hidden elements (512 bytes per row), copied with 16-byte cp.async by
+// all threads, so that kStages - 1 slabs of loads are in flight while one is
+// being used.  Warp (wt, we) of the CTA owns kTt tokens x kTe experts; lane l
+// of every warp keeps partial l of each of its pairs, i.e. the elements
+// h = 256 j + 8 l + i, taken with one fma each in increasing h, and the 32
+// partials are combined with the xor butterfly.  The result is the canonical
+// value for any tile shape.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(smem_dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+template <int kTt, int kTe, int kWt, int kWe, int kStages>
+struct StagedCfg {
+  static constexpr int kThreads = kWt * kWe * 32;
+  static constexpr int kRowsX = kWt * kTt;  // tokens per CTA
+  static constexpr int kRowsW = kWe * kTe;  // experts per CTA
+  static constexpr int kRows = kRowsX + kRowsW;
+  static constexpr int kStageBytes = kRows * 512;
+  static constexpr int kSmem = kStages * kStageBytes;
+  static_assert((kRows * 32) % kThreads == 0, "copy split");
+  static_assert(kTt * kTe <= 64, "pairs per warp");
+};
+
+// Two fp32 fmas in one instruction (each lane of the pair is an ordinary
+// round-to-nearest fma): d.{lo,hi} = a.{lo,hi} * b.{lo,hi} + d.{lo,hi}.
+__device__ __forceinline__ void fma2(uint64_t& d, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+
+template <int kTt, int kTe, int kWt, int kWe, int kStages, bool kPair>
+__global__ void __launch_bounds__(kWt * kWe * 32) router_logits_staged_kernel(const uint16_t* __restrict__ x,
+                                                                             const uint16_t* __restrict__ w_router,
+                                                                             const float* __restrict__ bias, int M,
+                                                                             int H, int E,
+                                                                             float* __restrict__ logits) {
+  using C = StagedCfg<kTt, kTe, kWt, kWe, kStages>;
+  extern __shared__ __align__(128) uint8_t slabs[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * kTokPerWarp;
-  const int e0 = (blockIdx.y * kWarps + warp) * kExp;
-  if (e0 >= E) return;
+  const int wt = warp / kWe, we = warp % kWe;
+  const int t_base = blockIdx.x * C::kRowsX, e_base = blockIdx.y * C::kRowsW;
+  const int nj = H / 256;
 
-  float acc[kTokPerWarp][kExp];
+  auto issue = [&](int j) {
+    uint8_t* st = slabs + (j % kStages) * C::kStageBytes;
 #pragma unroll
-  for (int t = 0; t < kTokPerWarp; ++t)
-#pragma unroll
-    for (int q = 0; q < kExp; ++q) acc[t][q] = 0.0f;
-
-  const int nchunk = H / 256;
-  uint4 wv[kExp], xv[kTokPerWarp];
-  auto load = [&](int j, uint4 (&wd)[kExp], uint4 (&xd)[kTokPerWarp]) {
-    const int h = 256 * j + 8 * lane;
-#pragma unroll
-    for (int q = 0; q < kExp; ++q)
-      wd[q] = (e0 + q < E) ? ld_nc_16(w_router + static_cast<size_t>(e0 + q) * H + h) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int t = 0; t < kTokPerWarp; ++t)
-      xd[t] = (t0 + t < M) ? ld_nc_16(x + static_cast<size_t>(t0 + t) * H + h) : make_uint4(0, 0, 0, 0);
+    for (int it = 0; it < C::kRows * 32 / C::kThreads; ++it) {
+      const int idx = threadIdx.x + it * C::kThreads;
+      const int r = idx >> 5, c = idx & 31;
+      const uint16_t* row;
+      bool valid;
+      if (r < C::kRowsX) {
+        valid = t_base + r < M;
+        row = x + static_cast<size_t>(valid ? t_base + r : 0) * H;
+      } else {
+        valid = e_base + r - C::kRowsX < E;
+        row = w_router + static_cast<size_t>(valid ? e_base + r - C::kRowsX : 0) * H;
+      }
+      cp_async_16(st + r * 512 + c * 16, row + 256 * j + 8 * c, valid ? 16 : 0);  // 0 bytes -> zero fill
+    }
   };
-  if (kPipe) load(0, wv, xv);
+
+  // kPair: the accumulators of tokens 2u and 2u+1 (same expert) share one
+  // 64-bit register and advance together in one paired fma.
+  static_assert(!kPair || kTt % 2 == 0, "token pairs");
+  float acc[kTt][kTe];
+  uint64_t acc2[kTt / 2][kTe];
+#pragma unroll
+  for (int t = 0; t < kTt; ++t)
+#pragma unroll
+    for (int q = 0; q < kTe; ++q) acc[t][q] = 0.0f;
+#pragma unroll
+  for (int u = 0; u < kTt / 2; ++u)
+#pragma unroll
+    for (int q = 0; q < kTe; ++q) acc2[u][q] = 0ull;
+
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < nj) issue(s);
+    cp_async_commit();
+  }
 #pragma unroll 1
-  for (int j = 0; j < nchunk; ++j) {
-    uint4 wn[kExp], xn[kTokPerWarp];
-    if (kPipe) {
-      if (j + 1 < nchunk) load(j + 1, wn, xn);
+  for (int j = 0; j < nj; ++j) {
+    if (j + kStages - 1 < nj) issue(j + kStages - 1);  // into the stage released at the end of j - 1
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();  // this thread's copies of slab j have landed
+    __syncthreads();               // and everyone else's
+    const uint8_t* st = slabs + (j % kStages) * C::kStageBytes;
+    uint4 xv[kTt], wv[kTe];
+#pragma unroll
+    for (int t = 0; t < kTt; ++t) xv[t] = *reinterpret_cast<const uint4*>(st + (wt * kTt + t) * 512 + lane * 16);
+#pragma unroll
+    for (int q = 0; q < kTe; ++q)
+      wv[q] = *reinterpret_cast<const uint4*>(st + (C::kRowsX + we * kTe + q) * 512 + lane * 16);
+    if (kPair) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {  // increasing h inside the chunk
+        uint64_t xp[kTt / 2], wp[kTe];
+#pragma unroll
+        for (int u = 0; u < kTt / 2; ++u) xp[u] = pack2(elem(xv[2 * u], i), elem(xv[2 * u + 1], i));
+#pragma unroll
+        for (int q = 0; q < kTe; ++q) {
+          const float w = elem(wv[q], i);
+          wp[q] = pack2(w, w);
+        }
+#pragma unroll
+        for (int u = 0; u < kTt / 2; ++u)
+#pragma unroll
+          for (int q = 0; q < kTe; ++q) fma2(acc2[u][q], xp[u], wp[q]);
+      }
     } else {
-      load(j, wv, xv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)  // increasing h inside the chunk
+#pragma unroll
+        for (int t = 0; t < kTt; ++t)
+#pragma unroll
+          for (int q = 0; q < kTe; ++q) acc[t][q] = __fmaf_rn(elem(xv[t], i), elem(wv[q], i), acc[t][q]);
     }
+    __syncthreads();  // the stage may be refilled
+  }
+  if (kPair) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)  // increasing h inside the chunk
+    for (int u = 0; u < kTt / 2; ++u)
 #pragma unroll
-      for (int t = 0; t < kTokPerWarp; ++t)
-#pragma unroll
-        for (int q = 0; q < kExp; ++q) acc[t][q] = __fmaf_rn(elem(xv[t], i), elem(wv[q], i), acc[t][q]);
-    if (kPipe && j + 1 < nchunk) {
-#pragma unroll
-      for (int q = 0; q < kExp; ++q) wv[q] = wn[q];
-#pragma unroll
-      for (int t = 0; t < kTokPerWarp; ++t) xv[t] = xn[t];
-    }
+      for (int q = 0; q < kTe; ++q) {
+        const float2 v = unpack2(acc2[u][q]);
+        acc[2 * u][q] = v.x;
+        acc[2 * u + 1][q] = v.y;
+      }
   }
 
 #pragma unroll
-  for (int t = 0; t < kTokPerWarp; ++t)
+  for (int t = 0; t < kTt; ++t)
 #pragma unroll
-    for (int q = 0; q < kExp; ++q) {
+    for (int q = 0; q < kTe; ++q) {
       float v = acc[t][q];
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
-      acc[t][q] = v;
-    }
-  // lane l stores pair l = (t, q) = (l / kExp, l % kExp)
-#pragma unroll
-  for (int t = 0; t < kTokPerWarp; ++t)
-#pragma unroll
-    for (int q = 0; q < kExp; ++q)
-      if (lane == t * kExp + q && t0 + t < M && e0 + q < E) {
-        const float b = bias != nullptr ? bias[e0 + q] : 0.0f;
-        logits[static_cast<size_t>(t0 + t) * E + e0 + q] = __fadd_rn(acc[t][q], b);
+      const int tok = t_base + wt * kTt + t, e = e_base + we * kTe + q;
+      if (lane == ((t * kTe + q) & 31) && tok < M && e < E) {
+        const float b = bias != nullptr ? bias[e] : 0.0f;
+        logits[static_cast<size_t>(tok) * E + e] = __fadd_rn(v, b);
       }
+    }
+}
+
+template <int kTt, int kTe, int kWt, int kWe, int kStages, bool kPair>
+cudaError_t launch_staged(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
+                          float* logits, cudaStream_t stream) {
+  using C = StagedCfg<kTt, kTe, kWt, kWe, kStages>;
+  auto kern = router_logits_staged_kernel<kTt, kTe, kWt, kWe, kStages, kPair>;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  static bool attr_set[64] = {};
+  if (C::kSmem > 48 * 1024 && dev < 64 && !attr_set[dev]) {
+    st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (st != cudaSuccess) return st;
+    attr_set[dev] = true;
+  }
+  dim3 grid((M + C::kRowsX - 1) / C::kRowsX, (E + C::kRowsW - 1) / C::kRowsW);
+  kern<<<grid, C::kThreads, C::kSmem, stream>>>(x, w_router, bias, M, H, E, logits);
+  return cudaGetLastError();
 }
 
 // (value, id) ordering of the selection: larger value first, then lower id.
@@ -255,15 +354,9 @@ __global__ void __launch_bounds__(128) router_topk_ext_kernel(const float* __res
 
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
                                  float* logits, cudaStream_t stream) {
-  const int tok_blocks = (M + kTokPerWarp - 1) / kTokPerWarp;
-  if (M <= 64) {  // few tokens: one expert per warp, so that enough warps stream W_r
-    dim3 grid(tok_blocks, (E + kWarps - 1) / kWarps);
-    router_logits_kernel<1, true><<<grid, kWarps * 32, 0, stream>>>(x, w_router, bias, M, H, E, logits);
-  } else {
-    dim3 grid(tok_blocks, (E + 4 * kWarps - 1) / (4 * kWarps));
-    router_logits_kernel<4, false><<<grid, kWarps * 32, 0, stream>>>(x, w_router, bias, M, H, E, logits);
-  }
-  return cudaGetLastError();
+  if (M <= 64)  // few tokens: one expert per warp, so that many warps share the reads of w_router; deep ring
+    return launch_staged<8, 1, 1, 4, 16, false>(x, w_router, bias, M, H, E, logits, stream);
+  return launch_staged<8, 8, 2, 2, 4, true>(x, w_router, bias, M, H, E, logits, stream);
 }
 
 cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t* topk_ids, float* topk_w,
