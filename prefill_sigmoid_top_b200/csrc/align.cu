@@ -23,19 +23,19 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 // Dynamic shared memory budget: the 227 KB per-block limit minus room for the
 // kernel's static shared variables.
 constexpr size_t kSmemLimit = 227 * 1024 - 1024;
 
-__global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restrict__ topk_ids, int n, int E, int B,
+template <int kWarps>
+__global__ void __launch_bounds__(kWarps * 32) align_kernel(const int32_t* __restrict__ topk_ids, int n, int E, int B,
                                                          int32_t* __restrict__ sorted_ids,
                                                          int32_t* __restrict__ block_expert,
                                                          int32_t* __restrict__ counts_out,
                                                          int32_t* __restrict__ offsets_out,
                                                          int32_t* __restrict__ ntpp_out, int32_t* err,
                                                          int stage_ids) {
+  constexpr int kThreads = kWarps * 32;
   extern __shared__ int smem[];
   int* hist = smem;                  // [kWarps][E]: counts, then write cursors
   int* prefix = hist + kWarps * E;   // [E + 1]
@@ -91,14 +91,14 @@ __global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restri
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int ws = warp_sums[lane];
+    const int ws = lane < kWarps ? warp_sums[lane] : 0;
     int wincl = ws;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, wincl, off);
       if (lane >= off) wincl += v;
     }
-    warp_sums[lane] = wincl - ws;  // exclusive prefix over warps
+    if (lane < kWarps) warp_sums[lane] = wincl - ws;  // exclusive prefix over warps
   }
   __syncthreads();
   const int excl = warp_sums[warp] + incl - padded;
@@ -157,12 +157,11 @@ __global__ void __launch_bounds__(kThreads) align_kernel(const int32_t* __restri
   }
 }
 
-}  // namespace
 
-cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, int32_t* sorted_ids,
-                         int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets, int32_t* ntpp,
-                         int32_t* err, cudaStream_t stream) {
-  const long long n = static_cast<long long>(M) * K;
+template <int kWarps>
+cudaError_t launch_align_variant(const int32_t* topk_ids, int n, int E, int B, int32_t* sorted_ids,
+                                 int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets,
+                                 int32_t* ntpp, int32_t* err, cudaStream_t stream) {
   const size_t base = sizeof(int) * (static_cast<size_t>(kWarps) * E + E + 1);
   const bool stage = base + sizeof(int) * static_cast<size_t>(n) <= kSmemLimit;
   const size_t smem = base + (stage ? sizeof(int) * static_cast<size_t>(n) : 0);
@@ -172,13 +171,30 @@ cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, in
   if (st != cudaSuccess) return st;
   static bool attr_set[64] = {};
   if (dev < 64 && !attr_set[dev]) {
-    st = cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemLimit));
+    st = cudaFuncSetAttribute(align_kernel<kWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kSmemLimit));
     if (st != cudaSuccess) return st;
     attr_set[dev] = true;
   }
-  align_kernel<<<1, kThreads, smem, stream>>>(topk_ids, M * K, E, B, sorted_ids, block_expert, expert_counts,
-                                             expert_offsets, ntpp, err, stage ? 1 : 0);
+  align_kernel<kWarps><<<1, kWarps * 32, smem, stream>>>(topk_ids, n, E, B, sorted_ids, block_expert, expert_counts,
+                                                       expert_offsets, ntpp, err, stage ? 1 : 0);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// One CTA; its thread count must cover the experts (one thread per expert in
+// the prefix step).  Few slots: 8 warps, so that the per-expert loops over
+// the warps' histogram rows are short; otherwise 32 warps.
+cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, int32_t* sorted_ids,
+                         int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets, int32_t* ntpp,
+                         int32_t* err, cudaStream_t stream) {
+  const int n = M * K;
+  if (n <= 4096 && E <= 256)
+    return launch_align_variant<8>(topk_ids, n, E, B, sorted_ids, block_expert, expert_counts, expert_offsets, ntpp,
+                                   err, stream);
+  return launch_align_variant<32>(topk_ids, n, E, B, sorted_ids, block_expert, expert_counts, expert_offsets, ntpp,
+                                  err, stream);
 }
 
 }  // namespace moe
