@@ -179,6 +179,29 @@ MOE_API moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weight
                                    moe_stream_t stream);
 MOE_API size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype);
 
+/* ------------------------------------------------------ self-routing up --
+ * moe_align_block_size and moe_grouped_up_swiglu in one launch (flashinfer
+ * PR #6511 analysis, §6: the align step folded into the first GEMM of the
+ * route chain, one launch fewer).  Every CTA of the up projection builds what
+ * it needs of the expert-major plan from topk_ids itself, computes its tile
+ * exactly as moe_grouped_up_swiglu does (32-row token tiles, x rows gathered
+ * by token id), and writes its part of the plan, so that on return the plan
+ * arrays hold exactly what moe_align_block_size writes and h exactly what
+ * moe_grouped_up_swiglu writes for that plan.
+ * x: bf16 [M,H]; w: MOE_W_BF16 weights; topk_ids: int32 [M,top_k] (device);
+ * plan outputs (device, sizes as moe_align_block_size); h: bf16 [cap, I];
+ * err_flag: device int32 (nullable), MOE_ERR_INVALID_INPUT if an id lies
+ * outside [0,E) (outputs then unspecified).
+ * Limit: M*top_k <= MOE_ROUTED_UP_MAX_SLOTS, else MOE_ERR_UNSUPPORTED;
+ * NVFP4 weights: MOE_ERR_UNSUPPORTED.  moe_layer takes this path by itself on
+ * decode shapes. */
+#define MOE_ROUTED_UP_MAX_SLOTS 1024
+MOE_API moe_status_t moe_grouped_up_swiglu_routed(const moe_bf16_t* x, const moe_weights_t* w,
+                                                  const int32_t* topk_ids, moe_shape_t s, int32_t* sorted_ids,
+                                                  int32_t* block_expert, int32_t* expert_counts,
+                                                  int32_t* expert_offsets, int32_t* num_tokens_post_padded,
+                                                  moe_bf16_t* h, int32_t* err_flag, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- down ---
  * Grouped down projection (flashinfer PR #6511 analysis, §1-§2).  For every
  * non-padding plan row r of expert e, with f = sorted_ids[r]:

@@ -99,6 +99,8 @@ def _declare(L):
         "moe_grouped_down": (st, [vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Plan), _Shape, vp, vp, sz, vp,
                                   vp]),
         "moe_down_workspace_size": (sz, [_Shape, ctypes.c_int]),
+        "moe_grouped_up_swiglu_routed": (st, [vp, ctypes.POINTER(_Weights), vp, _Shape, vp, vp, vp, vp, vp, vp, vp,
+                                              vp]),
         "moe_finalize_rmsnorm": (st, [vp, vp, vp, vp, ctypes.c_float, _Shape, vp, vp, vp]),
         "moe_layer": (st, [vp, vp, vp, ctypes.POINTER(_Weights), vp, ctypes.c_float, _Shape, vp, vp, vp, vp, vp,
                            sz, vp]),
@@ -270,6 +272,29 @@ def grouped_up_swiglu(x, w_gate, w_up, plan, shape: Shape, h=None, err_flag=None
                                            _ptr(ws), 0 if ws is None else ws.numel(), _ptr(err_flag), _stream()),
            "moe_grouped_up_swiglu")
     return h
+
+
+def grouped_up_swiglu_routed(x, w_gate, w_up, topk_ids, shape: Shape, h=None, plan=None, err_flag=None):
+    """Align + up projection in one launch: returns (h [cap, I] in plan order, plan dict of device tensors)."""
+    _need_cuda(x, w_gate, w_up, topk_ids)
+    cap = align_capacity(shape)
+    if cap == 0:
+        raise MoEError(2, "moe_align_capacity")
+    dev = x.device
+    if h is None:
+        h = torch.empty(cap, shape.I, dtype=torch.bfloat16, device=dev)
+    if plan is None:
+        plan = dict(sorted_ids=torch.empty(cap, dtype=torch.int32, device=dev),
+                    block_expert=torch.empty(cap // shape.block_size + 1, dtype=torch.int32, device=dev),
+                    expert_counts=torch.empty(shape.E, dtype=torch.int32, device=dev),
+                    expert_offsets=torch.empty(shape.E + 1, dtype=torch.int32, device=dev),
+                    num_tokens_post_padded=torch.empty(1, dtype=torch.int32, device=dev))
+    w = _weights_struct(w_gate, w_up, w_up)
+    _check(library().moe_grouped_up_swiglu_routed(
+        _ptr(_bf16(x)), ctypes.byref(w), _ptr(topk_ids), shape.c(), _ptr(plan["sorted_ids"]),
+        _ptr(plan["block_expert"]), _ptr(plan["expert_counts"]), _ptr(plan["expert_offsets"]),
+        _ptr(plan["num_tokens_post_padded"]), _ptr(h), _ptr(err_flag), _stream()), "moe_grouped_up_swiglu_routed")
+    return h, plan
 
 
 def grouped_down(h, w_down, plan, shape: Shape, y=None, err_flag=None):

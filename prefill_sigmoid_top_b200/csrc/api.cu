@@ -249,6 +249,44 @@ moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_
   return cuda_status(moe::launch_grouped_up(mg, mu, mx, a, choose_nmax(s), gathered, stream));
 }
 
+// Whether the layer folds the align step into the up projection: bf16
+// weights on the decode path (32-row token tiles, x gathered by token id) and
+// few enough routed slots for one warp per CTA to scan.  MOE_SELF_ROUTE=0
+// turns it off (the tests cover both).
+bool want_self_route(const moe_shape_t& s, moe_wdtype_t dt) {
+  if (const char* env = std::getenv("MOE_SELF_ROUTE"))
+    if (std::strcmp(env, "0") == 0) return false;
+  return dt == MOE_W_BF16 && !want_persistent(s) && choose_nmax(s) == 32 && !want_pregather(s) &&
+         static_cast<long long>(s.M) * s.top_k <= moe::kRouteMaxSlots;
+}
+
+moe_status_t run_up_routed(const moe_bf16_t* x, const moe_weights_t* w, const int32_t* topk_ids,
+                           const moe_shape_t& s, int32_t* sorted_ids, int32_t* block_expert, int32_t* counts,
+                           int32_t* offsets, int32_t* ntpp, moe_bf16_t* h, int32_t* err, cudaStream_t stream) {
+  CUtensorMap mg, mu, mx;
+  const uint64_t rows = static_cast<uint64_t>(s.E) * s.I;
+  if (!make_map_bf16(&mg, w->gate, rows, s.H, 128) || !make_map_bf16(&mu, w->up, rows, s.H, 128) ||
+      !make_map_bf16(&mx, x, s.M, s.H, 1))
+    return MOE_ERR_CUDA;
+  GroupedGemmArgs a{};
+  a.out = h;
+  a.err = err;
+  a.M = s.M;
+  a.E = s.E;
+  a.top_k = s.top_k;
+  a.rows_per_expert = s.I;
+  a.kdim = s.H;
+  a.out_ld = s.I;
+  a.topk_ids = topk_ids;
+  a.block_size = s.block_size;
+  a.plan_sorted_ids = sorted_ids;
+  a.plan_block_expert = block_expert;
+  a.plan_counts = counts;
+  a.plan_offsets = offsets;
+  a.plan_ntpp = ntpp;
+  return cuda_status(moe::launch_grouped_up_routed(mg, mu, mx, a, stream));
+}
+
 moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
                       moe_bf16_t* y, int32_t* err, cudaStream_t stream) {
   CUtensorMap md, mh;
@@ -501,6 +539,27 @@ moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, 
   return run_up(x, w, plan, s, h, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 
+static_assert(MOE_ROUTED_UP_MAX_SLOTS == moe::kRouteMaxSlots, "header and kernel agree on the slot limit");
+
+moe_status_t moe_grouped_up_swiglu_routed(const moe_bf16_t* x, const moe_weights_t* w, const int32_t* topk_ids,
+                                          moe_shape_t s, int32_t* sorted_ids, int32_t* block_expert,
+                                          int32_t* expert_counts, int32_t* expert_offsets,
+                                          int32_t* num_tokens_post_padded, moe_bf16_t* h, int32_t* err_flag,
+                                          moe_stream_t stream) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (w->dtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+  if ((st = check_weights(w, s)) != MOE_OK) return st;
+  if (static_cast<long long>(s.M) * s.top_k > moe::kRouteMaxSlots) return MOE_ERR_UNSUPPORTED;
+  if (!x || !topk_ids || !h || !w->gate || !w->up || !sorted_ids || !block_expert || !expert_counts ||
+      !expert_offsets || !num_tokens_post_padded)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(h) || !aligned16(w->gate) || !aligned16(w->up)) return MOE_ERR_INVALID_ARG;
+  return run_up_routed(x, w, topk_ids, s, sorted_ids, block_expert, expert_counts, expert_offsets,
+                       num_tokens_post_padded, h, err_flag, static_cast<cudaStream_t>(stream));
+}
+
 moe_status_t moe_grouped_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan, moe_shape_t s,
                               moe_bf16_t* y, void* ws, size_t ws_bytes, int32_t* err_flag, moe_stream_t stream) {
   moe_status_t st = check_shape(s);
@@ -576,10 +635,15 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
     return st;
   if ((st = cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, ids, tw, cs))) != MOE_OK) return st;
+  moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
+  if (want_self_route(s, w->dtype)) {
+    if ((st = run_up_routed(x, w, ids, s, sorted, bexp, counts, offs, ntpp, h, err, cs)) != MOE_OK) return st;
+    if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
+    return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
+  }
   if ((st = cuda_status(moe::launch_align(ids, s.M, s.top_k, s.E, s.block_size, sorted, bexp, counts, offs, ntpp,
                                           err, cs))) != MOE_OK)
     return st;
-  moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
   if (w->dtype == MOE_W_NVFP4) {
     uint8_t* act = base + L.act_scratch;
     if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs)) != MOE_OK) return st;

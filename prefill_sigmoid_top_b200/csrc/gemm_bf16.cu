@@ -33,6 +33,16 @@
 //                up:   h[row, i] = bf16(silu(gate) * up)   (fused SwiGLU)
 //                down: y[slot, j] = bf16(acc), scattered to the slot id.
 // Every wait is bounded; a timeout sets the error word and unwinds.
+//
+// Self-routing (kRoute, decode up only; flashinfer PR #6511 analysis, §6:
+// the align launch folded into the first GEMM of the chain): instead of
+// reading the plan, every CTA stages topk_ids (M*top_k <= kRouteMaxSlots) in
+// shared memory, counts the slots per expert, finds its tile as above, takes
+// the padded prefix of its expert and the slot ids of its token tile (one warp,
+// ascending slot order, ballots), and writes its part of the plan: the rows
+// and padding of its token tile (weight tile 0 only), and, in CTA 0, the
+// counts, offsets, block -> expert map and padded total.  The plan is the one
+// moe_align_block_size writes, bit for bit.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -68,7 +78,7 @@ struct Cfg {
 // kGatherB: the token rows of the B operand are gathered from x by token id
 // (tile::gather4); otherwise they are consecutive plan rows of a tensor that
 // is already in plan order (h, or x gathered by gather_rows_kernel).
-template <bool kUp, int kNmax, int kStages, bool kGatherB>
+template <bool kUp, int kNmax, int kStages, bool kGatherB, bool kRoute>
 __global__ void __launch_bounds__(128, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                         const __grid_constant__ CUtensorMap tm_b, const GroupedGemmArgs args) {
@@ -94,14 +104,63 @@ __global__ void __launch_bounds__(128, 1)
   // the token tiles that stream the same weight panel start together and the
   // panel is fetched from HBM once and shared through L2.
   int* cnt = reinterpret_cast<int*>(stages);  // scratch before the pipeline starts (E <= 1024)
-  for (int e = tid; e < E; e += 128) cnt[e] = args.expert_counts[e];
+  int* ids_s = cnt + 1024;                    // self-routing: topk_ids [M*top_k]
+  int* pre = ids_s + kRouteMaxSlots;          // self-routing, CTA 0: padded prefix [E+1]
+  int* slot_s = pre + 1025;                   // self-routing: slot ids of this token tile [kNmax]
+  const int nslots = args.M * args.top_k;
+  if (kRoute) {
+    for (int e = tid; e < E; e += 128) cnt[e] = 0;
+  } else {
+    for (int e = tid; e < E; e += 128) cnt[e] = args.expert_counts[e];
+  }
   if (tid == 0) {
     info[0] = -1;
     info[1] = 0;
     info[2] = 0;
+    info[3] = 0;
     *abort_flag = 0;
   }
   __syncthreads();
+  if (kRoute) {
+    for (int f = tid; f < nslots; f += 128) {
+      const int id = args.topk_ids[f];
+      ids_s[f] = id;
+      if (id >= 0 && id < E)
+        atomicAdd(&cnt[id], 1);
+      else
+        set_error(args.err, kErrInvalidInput);
+    }
+    __syncthreads();
+    const int B = args.block_size;
+    if (blockIdx.x == 0) {
+      // the plan header: counts, padded exclusive prefix, total, block -> expert
+      if (warp == 0) {
+        const int per = (E + 31) / 32;
+        const int lo = min(E, lane * per), hi = min(E, lo + per);
+        int sum = 0;
+        for (int e = lo; e < hi; ++e) sum += (cnt[e] + B - 1) / B * B;
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        int run = incl - sum;
+        for (int e = lo; e < hi; ++e) {
+          pre[e] = run;
+          run += (cnt[e] + B - 1) / B * B;
+        }
+        if (lane == 31) pre[E] = incl;
+      }
+      __syncthreads();
+      for (int e = tid; e <= E; e += 128) args.plan_offsets[e] = pre[e];
+      for (int e = tid; e < E; e += 128) {
+        args.plan_counts[e] = cnt[e];
+        for (int b = pre[e] / B; b < pre[e + 1] / B; ++b) args.plan_block_expert[b] = e;
+      }
+      if (tid == 0) *args.plan_ntpp = pre[E];
+    }
+  }
   if (warp == 0) {
     const int linear = blockIdx.x;
     const int per = (E + 31) / 32;
@@ -137,13 +196,48 @@ __global__ void __launch_bounds__(128, 1)
   const int wt = info[2];
   const int count_e = cnt[e];
   const int nrows = min(kNmax, count_e - local * kNmax);
-  const int row0 = args.expert_offsets[e] + local * kNmax;
+  if (kRoute) {
+    const int B = args.block_size;
+    if (warp == 0) {
+      // padded offset of expert e
+      const int per = (E + 31) / 32;
+      const int lo = min(e, lane * per), hi = min(e, lo + per);
+      int sum = 0;
+      for (int q = lo; q < hi; ++q) sum += (cnt[q] + B - 1) / B * B;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane == 0) info[3] = sum;
+      // slot ids of token tile `local` of expert e, in ascending slot order
+      const unsigned lt_mask = (1u << lane) - 1u;
+      const int first = local * kNmax;
+      int seen = 0;
+      for (int base = 0; base < nslots && seen < first + nrows; base += 32) {
+        const int f = base + lane;
+        const bool m = f < nslots && ids_s[f] == e;
+        const unsigned bal = __ballot_sync(0xffffffffu, m);
+        const int pos = seen + __popc(bal & lt_mask);
+        if (m && pos >= first && pos < first + nrows) slot_s[pos - first] = f;
+        seen += __popc(bal);
+      }
+    }
+    __syncthreads();
+  }
+  const int off_e = kRoute ? info[3] : args.expert_offsets[e];
+  const int row0 = off_e + local * kNmax;
   const int N = (nrows + 15) & ~15;
-  const int nslots = args.M * args.top_k;
+  if (kRoute && wt == 0) {
+    // this token tile's rows of the plan, and the expert's padding after its last tile
+    for (int n = tid; n < nrows; n += 128) args.plan_sorted_ids[row0 + n] = slot_s[n];
+    if (local == (count_e - 1) / kNmax) {
+      const int B = args.block_size;
+      const int pad_end = off_e + (count_e + B - 1) / B * B;
+      for (int p = off_e + count_e + tid; p < pad_end; p += 128) args.plan_sorted_ids[p] = nslots;
+    }
+  }
   for (int n = tid; n < N; n += 128) {
     int v = (kUp && kGatherB) ? 0 : -1;
     if (n < nrows) {
-      const int id = args.sorted_ids[row0 + n];
+      const int id = kRoute ? slot_s[n] : args.sorted_ids[row0 + n];
       if (id >= 0 && id < nslots) {
         v = (kUp && kGatherB) ? id / args.top_k : id;
       } else {
@@ -308,11 +402,14 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <bool kUp, int kNmax, int kStages, bool kGatherB>
+template <bool kUp, int kNmax, int kStages, bool kGatherB, bool kRoute = false>
 cudaError_t launch_variant(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                            const GroupedGemmArgs& args, cudaStream_t stream) {
   using C = Cfg<kUp, kNmax, kStages>;
-  auto kern = grouped_gemm_kernel<kUp, kNmax, kStages, kGatherB>;
+  static_assert(!kRoute || (kUp && kGatherB), "self-routing: up projection with gathered x rows only");
+  static_assert(!kRoute || (1024 + kRouteMaxSlots + 1025 + kNmax) * 4 <= kStages * C::kStageBytes,
+                "self-routing scratch fits in the stage buffers");
+  auto kern = grouped_gemm_kernel<kUp, kNmax, kStages, kGatherB, kRoute>;
   int dev = 0;
   cudaError_t st = cudaGetDevice(&dev);
   if (st != cudaSuccess) return st;
@@ -356,6 +453,12 @@ cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up
   if (nmax <= 32) return launch_variant<true, 32, 3, true>(w_gate, w_up, x_rows, args, stream);
   if (nmax <= 128) return launch_variant<true, 128, 2, true>(w_gate, w_up, x_rows, args, stream);
   return launch_variant<true, 256, 3, true>(w_gate, w_up, x_rows, args, stream);
+}
+
+cudaError_t launch_grouped_up_routed(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                                     const GroupedGemmArgs& args, cudaStream_t stream) {
+  if (args.M * args.top_k > kRouteMaxSlots || args.E > 1024) return cudaErrorInvalidValue;
+  return launch_variant<true, 32, 3, true, true>(w_gate, w_up, x_rows, args, stream);
 }
 
 cudaError_t launch_grouped_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,

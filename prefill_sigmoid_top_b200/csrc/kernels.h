@@ -47,7 +47,20 @@ struct GroupedGemmArgs {
   int rows_per_expert; // up: I; down: H  (weight rows of one expert)
   int kdim;            // up: H; down: I  (contraction length)
   int out_ld;          // up: I; down: H
+  // Self-routing up only (null otherwise): the routed ids it reads instead of
+  // the plan, and the plan it writes for the kernels that follow.
+  const int32_t* topk_ids;
+  int block_size;
+  int32_t* plan_sorted_ids;
+  int32_t* plan_block_expert;
+  int32_t* plan_counts;
+  int32_t* plan_offsets;
+  int32_t* plan_ntpp;
 };
+
+// Largest M*top_k the self-routing up kernel accepts (the ids are staged in
+// shared memory and scanned by one warp per CTA).
+constexpr int kRouteMaxSlots = 1024;
 
 // `nmax` selects the token-tile width (32 or 128).  Tensor maps: a0/a1 are
 // the weight matrices viewed as 2-D [E*rows_per_expert, kdim]; b is x [M,H]
@@ -59,6 +72,11 @@ cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up
 // xg[r] = x[sorted_ids[r] / top_k] for the real plan rows r < ntpp.
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* sorted_ids, const int32_t* ntpp, int M, int top_k,
                                int H, int cap, uint16_t* xg, cudaStream_t stream);
+// Decode up projection that builds the plan itself from topk_ids (32-row
+// token tiles, x rows gathered by token id) and writes it for the down and
+// finalize kernels: the align step folded into the up kernel.
+cudaError_t launch_grouped_up_routed(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                                     const GroupedGemmArgs& args, cudaStream_t stream);
 cudaError_t launch_grouped_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
                                 int nmax, cudaStream_t stream);
 

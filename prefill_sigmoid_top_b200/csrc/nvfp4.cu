@@ -240,17 +240,19 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(
 // x enters the up projection once per routed slot, i.e. up to top_k times per
 // token, so it is quantised once per token (quantize_kernel) and this kernel
 // copies each slot's codes and scales into the tile-aligned layout: token tile
-// `blockIdx.x`, row r <- token sorted_ids[row0 + r] / top_k.  One warp per row;
-// a row's scales (cols/16 bytes) move as 4-byte words, each word the four
-// column blocks of one scale atom row.  Rows past the expert's count are not
-// written (as above).
+// `blockIdx.x`, row r <- token sorted_ids[row0 + r] / top_k.  The tile's token
+// ids are staged in shared memory first; then every thread copies independent
+// 16-byte code chunks and 4-byte scale words (four column blocks of one scale
+// atom row), so many loads are in flight.  Rows past the expert's count are
+// not written (as above).
 __global__ void __launch_bounds__(256) gather_tiles_kernel(
     const uint8_t* __restrict__ tok_codes, const uint8_t* __restrict__ tok_scales,
     const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
     int E, int top_k, int nslots, int cols, uint8_t* __restrict__ codes, uint8_t* __restrict__ atoms) {
   __shared__ int s_cnt[1024];
   __shared__ int s_info[2];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int s_tok[128];
+  const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = counts[e];
   __syncthreads();
   const int ti = blockIdx.x;
@@ -260,19 +262,28 @@ __global__ void __launch_bounds__(256) gather_tiles_kernel(
   const int local = s_info[1];
   const int nrows = min(128, s_cnt[e] - local * 128);
   const int row0 = offsets[e] + local * 128;
+  for (int r = tid; r < nrows; r += blockDim.x) {
+    const int id = sorted_ids[row0 + r];
+    s_tok[r] = (id >= 0 && id < nslots) ? id / top_k : -1;
+  }
+  __syncthreads();
   const int cb16 = cols / 32;  // 16-byte code chunks per row
   const int nw = cols / 64;    // scale words per row
-  for (int r = warp; r < nrows; r += blockDim.x / 32) {
-    const int id = sorted_ids[row0 + r];
-    const int t = (id >= 0 && id < nslots) ? id / top_k : -1;
-    const uint4* src = reinterpret_cast<const uint4*>(tok_codes + static_cast<int64_t>(t < 0 ? 0 : t) * (cols / 2));
-    uint4* dst = reinterpret_cast<uint4*>(codes + (static_cast<int64_t>(ti) * 128 + r) * (cols / 2));
-    for (int c = lane; c < cb16; c += 32) dst[c] = t >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
-    const uint32_t* ssrc =
-        reinterpret_cast<const uint32_t*>(tok_scales + static_cast<int64_t>(t < 0 ? 0 : t) * (cols / 16));
-    for (int a = lane; a < nw; a += 32)
-      *reinterpret_cast<uint32_t*>(atoms + (static_cast<int64_t>(ti) * nw + a) * 512 + (r % 32) * 16 + (r / 32) * 4) =
-          t >= 0 ? ssrc[a] : 0u;
+  const uint4* src = reinterpret_cast<const uint4*>(tok_codes);
+  uint4* dst = reinterpret_cast<uint4*>(codes) + static_cast<int64_t>(ti) * 128 * cb16;
+#pragma unroll 4
+  for (int i = tid; i < nrows * cb16; i += blockDim.x) {
+    const int r = i / cb16, c = i - r * cb16;
+    const int t = s_tok[r];
+    dst[static_cast<int64_t>(r) * cb16 + c] = t >= 0 ? src[static_cast<int64_t>(t) * cb16 + c] : make_uint4(0, 0, 0, 0);
+  }
+  const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(tok_scales);
+#pragma unroll 4
+  for (int i = tid; i < nrows * nw; i += blockDim.x) {
+    const int r = i / nw, a = i - r * nw;
+    const int t = s_tok[r];
+    *reinterpret_cast<uint32_t*>(atoms + (static_cast<int64_t>(ti) * nw + a) * 512 + (r % 32) * 16 + (r / 32) * 4) =
+        t >= 0 ? ssrc[static_cast<int64_t>(t) * nw + a] : 0u;
   }
 }
 

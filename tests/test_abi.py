@@ -127,3 +127,20 @@ def test_route_ex_rejects_bad_options():
     assert L.moe_route_ex(*args(ctypes.byref(_RouteOpts(1, 1, 1, float("nan"))))) == 1
     assert L.moe_route_ex(FAKE, FAKE, None, s, ctypes.byref(ok), FAKE, FAKE, FAKE, 4, None) == 3
     assert L.moe_route_ex(FAKE_MIS, FAKE, None, s, ctypes.byref(ok), FAKE, FAKE, FAKE, 1 << 20, None) == 1
+
+
+def test_routed_up_rejects_bad_arguments():
+    L = moe.library()
+    w = _Weights(0, 0x10000, 0x10000, 0x10000, None, None, None)
+    args = lambda shape, wp: (FAKE, wp, FAKE, shape.c(), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None)
+    big = moe.Shape(M=129, H=256, I=128, E=8, top_k=8, block_size=16)  # 1032 slots > 1024
+    assert L.moe_grouped_up_swiglu_routed(*args(big, ctypes.byref(w))) == 2
+    w_nv = _Weights(1, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert L.moe_grouped_up_swiglu_routed(*args(C0, ctypes.byref(w_nv))) == 2
+    assert L.moe_grouped_up_swiglu_routed(*args(C0, None)) == 1
+    a = list(args(C0, ctypes.byref(w)))
+    a[0] = FAKE_MIS
+    assert L.moe_grouped_up_swiglu_routed(*a) == 1
+    a = list(args(C0, ctypes.byref(w)))
+    a[4] = None
+    assert L.moe_grouped_up_swiglu_routed(*a) == 1
