@@ -239,6 +239,11 @@ MOE_API moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, 
                        void* ws, size_t ws_bytes, moe_stream_t stream);
 MOE_API size_t moe_layer_workspace_size(moe_shape_t s, moe_wdtype_t dtype);
 
+/* Number of kernels one moe_layer call launches for this shape and weight
+ * type (the stream-ordered memsets of its error and scale words not counted);
+ * -1 for an unsupported shape or dtype.  Host only, no CUDA call. */
+MOE_API int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype);
+
 /* Byte offsets of the layer's intermediates inside ws (for inspection). */
 typedef struct {
   size_t err_flag, logits, topk_ids, topk_w, sorted_ids, block_expert, expert_counts, expert_offsets,

@@ -105,6 +105,7 @@ def _declare(L):
         "moe_layer": (st, [vp, vp, vp, ctypes.POINTER(_Weights), vp, ctypes.c_float, _Shape, vp, vp, vp, vp, vp,
                            sz, vp]),
         "moe_layer_workspace_size": (sz, [_Shape, ctypes.c_int]),
+        "moe_layer_kernel_count": (ctypes.c_int, [_Shape, ctypes.c_int]),
         "moe_layer_workspace_layout": (st, [_Shape, ctypes.c_int, ctypes.POINTER(_Layout)]),
         "moe_quantize_nvfp4": (st, [vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, vp, vp, vp, vp, sz, vp]),
         "moe_nvfp4_quantize_workspace_size": (sz, [ctypes.c_int64]),
@@ -252,6 +253,11 @@ def align_block_size(topk_ids, E, block_size, err_flag=None, out=None):
 def _plan_struct(plan):
     return _Plan(plan["sorted_ids"].data_ptr(), plan["block_expert"].data_ptr(), plan["expert_counts"].data_ptr(),
                  plan["expert_offsets"].data_ptr(), plan["num_tokens_post_padded"].data_ptr())
+
+
+def layer_kernel_count(shape: Shape, wdtype: int = MOE_W_BF16) -> int:
+    """Kernels one moe_layer call launches for this shape (host-side count)."""
+    return int(library().moe_layer_kernel_count(shape.c(), wdtype))
 
 
 def up_workspace_size(shape: Shape, wdtype: int = MOE_W_BF16) -> int:

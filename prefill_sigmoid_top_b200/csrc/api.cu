@@ -655,6 +655,14 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
 }
 
+int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype) {
+  if (check_shape(s) != MOE_OK || (dtype != MOE_W_BF16 && dtype != MOE_W_NVFP4)) return -1;
+  if (dtype == MOE_W_NVFP4)  // router x2, align, amax, quantize x, gather tiles, up, amax h, quantize h, down, finalize
+    return 11;
+  if (want_self_route(s, dtype)) return 5;  // router x2, up with the plan, down, finalize
+  return 6 + (want_pregather(s) ? 1 : 0);   // router x2, align, [gather x], up, down, finalize
+}
+
 moe_status_t moe_quantize_nvfp4(const moe_bf16_t* src, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* codes,
                                 uint8_t* scales, float* gs, void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (n_mats < 1 || rows < 1 || cols < 16 || cols % 16 != 0) return MOE_ERR_UNSUPPORTED;

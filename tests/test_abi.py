@@ -144,3 +144,11 @@ def test_routed_up_rejects_bad_arguments():
     a = list(args(C0, ctypes.byref(w)))
     a[4] = None
     assert L.moe_grouped_up_swiglu_routed(*a) == 1
+
+
+def test_layer_kernel_count():
+    assert moe.layer_kernel_count(C1) == 5            # decode: align folded into the up kernel
+    batch = moe.Shape(M=512, H=7168, I=2048, E=256, top_k=16, block_size=64)
+    assert moe.layer_kernel_count(batch) == 7         # align and a gather pass of x
+    assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 11
+    assert moe.layer_kernel_count(moe.Shape(M=16, H=255, I=128, E=8, top_k=2, block_size=16)) == -1
