@@ -309,6 +309,29 @@ def run_ours(args):
     if moe.get_device_error(ws[eo:eo + 4].view(torch.int32)) != 0:
         raise SystemExit("device error in the timed layer calls")
 
+    # ---- the same call replayed from a CUDA graph (launch work taken off the host)
+    graph_ms = None
+    if world == 1:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer_step(d["x"], out_layer)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer_step(d["x"], out_layer)
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = g0.elapsed_time(g1) / args.steps
+        del graph
+
     # ---- end to end through the public entry point (moe_layer) with host buffers
     x_host = d["x"].cpu().pin_memory()
     out_host = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16).pin_memory()
@@ -367,6 +390,7 @@ def run_ours(args):
                    "l2": "no flush: each step streams GBs of expert weights, far above the 126 MB L2"},
         "kernels_us": {s: v * 1e3 for s, v in stage_ms.items()},
         "staged_us_per_layer": staged_ms * 1e3,
+        "graph_us_per_layer": None if graph_ms is None else graph_ms * 1e3,
         "gpu_launches": moe.layer_kernel_count(shape, wdt) * args.steps,
         "roofline": {"bound": "hbm", "kernel": "grouped_up_swiglu", "achieved": achieved, "peak": hbm_peak,
                      "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,

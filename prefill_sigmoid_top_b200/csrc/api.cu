@@ -207,10 +207,14 @@ moe_status_t check_weights(const moe_weights_t* w, const moe_shape_t& s) {
 }
 
 // NVFP4 up: amax of x -> tile-aligned NVFP4 copy of the routed x rows -> block-scaled GEMM.
+// h_amax (nullable): word the up epilogue atomically maxes |h| into (the caller zeroes it first).
 moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
-                          const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream);
+                          const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream,
+                          unsigned* h_amax = nullptr);
+// amax_ready: ws's amax word already holds max |h| (from the up epilogue); otherwise it is computed here.
 moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
-                            const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream);
+                            const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream,
+                            bool amax_ready = false);
 
 moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
                     moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t stream) {
@@ -314,7 +318,8 @@ moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_pla
 int num_sms();
 
 moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
-                          const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream) {
+                          const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream,
+                          unsigned* h_amax) {
   const ActLayout L = x_act_layout(s);
   auto* base = static_cast<uint8_t*>(ws);
   auto* amax = reinterpret_cast<unsigned*>(base + L.amax);
@@ -350,19 +355,23 @@ moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe
   a.gs_a0 = w->gate_gs;
   a.gs_a1 = w->up_gs;
   a.act_amax = amax;
+  a.out_amax = h_amax;
   return cuda_status(moe::launch_nvfp4_up(mg, mu, mx, a, num_sms(), stream));
 }
 
 moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
-                            const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream) {
+                            const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream,
+                            bool amax_ready) {
   const ActLayout L = h_act_layout(s);
   auto* base = static_cast<uint8_t*>(ws);
   auto* amax = reinterpret_cast<unsigned*>(base + L.amax);
   const int tiles = nvfp4_tiles_ub(s);
-  if (cudaMemsetAsync(amax, 0, sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (moe::launch_amax_plan_rows(h, plan->sorted_ids, plan->num_tokens_post_padded, s.M * s.top_k, s.I,
-                                 static_cast<int>(cap_rows(s)), amax, stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (!amax_ready) {
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::launch_amax_plan_rows(h, plan->sorted_ids, plan->num_tokens_post_padded, s.M * s.top_k, s.I,
+                                   static_cast<int>(cap_rows(s)), amax, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (moe::launch_quantize_tiles(h, plan->expert_counts, plan->expert_offsets, s.E, s.I, tiles, amax, base + L.codes,
                                  base + L.atoms, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -645,9 +654,13 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
                                           err, cs))) != MOE_OK)
     return st;
   if (w->dtype == MOE_W_NVFP4) {
+    // max |h| comes out of the up kernel's epilogue into the down activation copy's amax word
     uint8_t* act = base + L.act_scratch;
-    if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs)) != MOE_OK) return st;
-    if ((st = run_down_nvfp4(h, w, &plan, s, y, act + x_act_layout(s).total, err, cs)) != MOE_OK) return st;
+    uint8_t* act_h = act + x_act_layout(s).total;
+    auto* h_amax = reinterpret_cast<unsigned*>(act_h + h_act_layout(s).amax);
+    if ((st = cuda_status(cudaMemsetAsync(h_amax, 0, sizeof(unsigned), cs))) != MOE_OK) return st;
+    if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs, h_amax)) != MOE_OK) return st;
+    if ((st = run_down_nvfp4(h, w, &plan, s, y, act_h, err, cs, true)) != MOE_OK) return st;
   } else {
     if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
     if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
@@ -657,8 +670,8 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
 
 int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK || (dtype != MOE_W_BF16 && dtype != MOE_W_NVFP4)) return -1;
-  if (dtype == MOE_W_NVFP4)  // router x2, align, amax, quantize x, gather tiles, up, amax h, quantize h, down, finalize
-    return 11;
+  if (dtype == MOE_W_NVFP4)  // router x2, align, amax x, quantize x, gather tiles, up (+ amax h), quantize h, down, finalize
+    return 10;
   if (want_self_route(s, dtype)) return 5;  // router x2, up with the plan, down, finalize
   return 6 + (want_pregather(s) ? 1 : 0);   // router x2, align, [gather x], up, down, finalize
 }

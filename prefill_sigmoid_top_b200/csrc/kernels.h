@@ -101,6 +101,7 @@ struct Nvfp4GemmArgs {
   const float* gs_a0;     // [E] global scales of the tm_a0 matrix
   const float* gs_a1;     // [E]
   const unsigned* act_amax;  // activation amax (fp32 bits); gs = amax / 2688
+  unsigned* out_amax;        // up only, nullable: max |h| over the h values written (fp32 bits, atomic max)
 };
 
 // Quantise n_mats matrices [rows, cols] (bf16, back to back) to NVFP4 codes /

@@ -529,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 4) >> 2;
     const float act_gs = nvfp4_global_scale(__uint_as_float(*args.act_amax));
+    float hmax = 0.0f;  // up: max |h| of the values this thread stores
     int j = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
       const TileCoord c = decode_tile(prefix, cnt, E, tile);
@@ -583,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float gt = __uint_as_float(v0[i][qq]) * s0;
               const float ut = __uint_as_float(v1[i][qq]) * s1;
               const int col = c.w * kBM + q * 32 + lane;
-              out[static_cast<size_t>(row0 + n) * g.out_ld + col] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * ut);
+              const __nv_bfloat16 hv = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * ut);
+              out[static_cast<size_t>(row0 + n) * g.out_ld + col] = hv;
+              hmax = fmaxf(hmax, fabsf(__bfloat162float(hv)));
             }
           } else {
             const int id = __shfl_sync(0xffffffffu, id_word, (cb & 31) + qq);
@@ -596,6 +599,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+    }
+    if (kUp && args.out_amax != nullptr) {
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, off));
+      if (lane == 0 && hmax > 0.0f) atomicMax(args.out_amax, __float_as_uint(hmax));
     }
   }
   tc_fence_before_sync();

@@ -150,5 +150,5 @@ def test_layer_kernel_count():
     assert moe.layer_kernel_count(C1) == 5            # decode: align folded into the up kernel
     batch = moe.Shape(M=512, H=7168, I=2048, E=256, top_k=16, block_size=64)
     assert moe.layer_kernel_count(batch) == 7         # align and a gather pass of x
-    assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 11
+    assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 10
     assert moe.layer_kernel_count(moe.Shape(M=16, H=255, I=128, E=8, top_k=2, block_size=16)) == -1
