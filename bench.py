@@ -455,11 +455,13 @@ def run_reference(args):
     import numpy as np
     import torch
     import oracle
+    from prefill_sigmoid_top_b200 import inputs
     cfg = workload(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     d = inputs.make_inputs(cfg, dev)
     x, wr, b, g, wg, wu, wd = _oracle_host_inputs(cfg, d)
     del d
+    touched = int(len(set(int(e) for e in oracle.route(x, wr, b, cfg.K)[0].ravel())))
     # size one step so that the whole run stays within a few minutes
     t0 = time.perf_counter()
     oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=np.arange(1, dtype=np.int32))
@@ -482,7 +484,9 @@ def run_reference(args):
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": cfg.name, "M": cfg.M, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.K,
-                   "block_size": cfg.B, "seed": cfg.seed},
+                   "block_size": cfg.B, "seed": cfg.seed, "router_bias": cfg.bias, "touched_experts": touched,
+                   "parallelism": "host cores (CPU oracle)",
+                   "l2": "no flush: each step streams GBs of expert weights, far above the 126 MB L2"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
