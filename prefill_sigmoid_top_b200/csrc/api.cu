@@ -216,6 +216,20 @@ moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const m
                             const moe_shape_t& s, moe_bf16_t* y, void* ws, int32_t* err, cudaStream_t stream,
                             bool amax_ready = false);
 
+// Token-tile width of the 2-SM pair kernels on the persistent path, or 0 for
+// the single-SM persistent kernels.  Pairs measured faster on the batch and
+// prefill workloads (the operand feed per SM is the limit there): 256-row
+// tiles from 96 routed rows per expert on average, 128-row tiles below.
+// MOE_GEMM_PAIR=0|128|256 overrides (the tests cover every variant).
+int pair_nmax(const moe_shape_t& s) {
+  if (const char* env = std::getenv("MOE_GEMM_PAIR")) {
+    const int v = std::atoi(env);
+    return (v == 128 || v == 256) ? v : 0;
+  }
+  const double per_expert = static_cast<double>(s.M) * s.top_k / s.E;
+  return per_expert >= 96.0 ? 256 : 128;
+}
+
 moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
                     moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t stream) {
   CUtensorMap mg, mu, mx;
@@ -247,6 +261,8 @@ moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_
   a.rows_per_expert = s.I;
   a.kdim = s.H;
   a.out_ld = s.I;
+  if (persistent && gathered && pair_nmax(s) != 0 && s.I % 256 == 0)
+    return cuda_status(moe::launch_pair_up(mg, mu, mx, a, pair_nmax(s), num_sms(), stream));
   if (persistent)
     return cuda_status(
         moe::launch_persistent_up(mg, mu, mx, a, choose_nmax(s), !gathered, deep_token_ring(), num_sms(), stream));
@@ -310,6 +326,8 @@ moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_pla
   a.rows_per_expert = s.H;
   a.kdim = s.I;
   a.out_ld = s.H;
+  if (persistent && pair_nmax(s) != 0 && s.H % 512 == 0)
+    return cuda_status(moe::launch_pair_down(md, mh, a, pair_nmax(s), num_sms(), stream));
   if (persistent)
     return cuda_status(moe::launch_persistent_down(md, mh, a, choose_nmax(s), deep_token_ring(), num_sms(), stream));
   return cuda_status(moe::launch_grouped_down(md, mh, a, choose_nmax(s), stream));

@@ -1,0 +1,477 @@
+// Grouped expert projections on 2-SM pairs for batch and prefill shapes
+// ("[flashinfer] ... AlphaMoE NVFP4 커널 최적화", flashinfer PR #6511 analysis:
+// the up / down kernels of the route chain, §6; wide weight panels streamed by
+// TMA, §2).
+//
+// Why: with one CTA per SM and 128-row token tiles the persistent kernel is
+// bound by the operand feed into shared memory (each SM reads its weight tile
+// and all the token rows of its tile for every stage).  Here two CTAs of a
+// cluster run one tcgen05.mma.cta_group::2 of M = 256 weight rows: each CTA
+// holds 128 weight rows (A) and half of the token rows (B) of the tile in its
+// own shared memory, and each CTA's tensor memory receives its 128 rows of the
+// product for all N tokens.  Per SM the token-row bytes per flop halve, and a
+// token tile covers twice the weight rows per MMA instruction.
+//
+// Pair protocol (CTA rank 0 = leader, rank 1 = peer):
+//   * both CTAs allocate tensor memory together (cta_group::2, same warp);
+//   * each CTA's producers wait on their own "empty" barriers and load their
+//     own halves; all copies complete on the leader's "full" barriers, for
+//     which the leader alone posts the expected bytes of both CTAs;
+//   * the leader's one MMA thread waits on its full barriers, issues the
+//     MMAs, and its commits arrive on the empty barriers of both CTAs (the
+//     commit's CTA mask) and on both CTAs' accumulator-full barriers;
+//   * each CTA's epilogue drains its own tensor memory and arrives on the
+//     leader's accumulator-empty barrier (the peer's arrive remotely).
+// Copies are plain TMA loads with cta_group::2 (no multicast).
+//
+// Tiles: (expert e, weight block w, token tile t) over a static round-robin
+// list of tiles per pair, ordered e, w, t.  A token tile holds up to kNmax
+// plan rows; N = rows rounded up to 16; CTA r loads plan rows [r N/2, (r+1) N/2).
+//   up:   weight block w = rows 256w..256w+255 of W_gate and of W_up; CTA r
+//         holds rows 256w + 128r..+127 of both; h[row, 256w + 128r + i] =
+//         bf16(silu(gate) * up) from its two accumulators.
+//   down: weight block w = rows 512w..512w+511 of W_down as two M = 256
+//         halves; CTA r holds rows 512w + 128r.. and 512w + 256 + 128r..;
+//         y[slot, col] = bf16(acc), scattered to the slot.
+// Warp roles (384 threads per CTA): 0 = weight producer, 1 = MMA issuer
+// (leader only), 2 = token-row producer, 3 = idle, 4..11 = epilogue.
+// All mbarrier waits are bounded; a timeout sets the error word and unwinds,
+// and both CTAs still meet at the final cluster barrier.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;                  // weight rows per CTA (MMA M = 256 per pair)
+constexpr int kBK = 64;                   // contraction elements per stage
+constexpr int kBoxBytes = kBM * kBK * 2;  // one 128 x 64 bf16 box: 16 KB
+constexpr int kBRows = 32;                // rows per token-row box
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 128 + 32 * kEpiWarps;
+
+template <int kNmax, int kStagesA, int kStagesB>
+struct QCfg {
+  static constexpr int kHalf = kNmax / 2;  // token rows per CTA
+  static constexpr int kAStage = 2 * kBoxBytes;
+  static constexpr int kBStage = kHalf * kBK * 2;
+  static constexpr int kAccCols = 2 * kNmax;
+  static constexpr int kAccBufs = 512 / kAccCols;
+  static constexpr int kMisc = 10240;  // barriers, flags, counts and tile prefix over experts (E <= 1024)
+  static constexpr int kSmem = 1024 + kStagesA * kAStage + kStagesB * kBStage + kMisc;
+  static_assert(kNmax == 128 || kNmax == 256, "pair token-tile widths");
+  static_assert(kHalf % kBRows == 0, "whole token-row boxes per CTA");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kSmem > 116 * 1024, "one CTA per SM: it owns all 512 tensor-memory columns");
+};
+
+// ---------------------------------------------------------------- pair PTX
+__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+// 2-D tiled load into this CTA's shared memory; the bytes complete on the
+// mbarrier at cluster address `bar` (the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar, void* dst, int32_t c0,
+                                                 int32_t c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D (+)= A * B^T over the pair: M = 256 (128 rows of A in each CTA), B rows
+// split between the CTAs, D rows split between their tensor memories.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive (once the pair's earlier tcgen05 work has completed) on the mbarrier
+// at this shared-memory offset in both CTAs of the pair.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+struct TileCoord {
+  int e, w, t;
+};
+
+template <int kNmax>
+__device__ __forceinline__ TileCoord decode_tile(const int* prefix, const int* cnt, int E, int idx) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= idx) lo = mid; else hi = mid - 1;
+  }
+  const int ntiles = (cnt[lo] + kNmax - 1) / kNmax;
+  const int rel = idx - prefix[lo];
+  return TileCoord{lo, rel / ntiles, rel % ntiles};
+}
+
+template <int kN>
+__device__ __forceinline__ int pick(const int (&ids)[kN], int i) {
+  int v = ids[0];
+#pragma unroll
+  for (int j = 1; j < kN; ++j) v = (i == j) ? ids[j] : v;
+  return v;
+}
+
+template <bool kUp, int kNmax, int kStagesA, int kStagesB>
+__global__ void __launch_bounds__(kThreads, 1)
+    pair_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
+                     const __grid_constant__ CUtensorMap tm_b, const GroupedGemmArgs args) {
+  using C = QCfg<kNmax, kStagesA, kStagesB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_ring = smem;
+  uint8_t* b_ring = a_ring + kStagesA * C::kAStage;
+  uint8_t* misc = b_ring + kStagesB * C::kBStage;
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* a_empty = a_full + kStagesA;
+  uint64_t* b_full = a_empty + kStagesA;
+  uint64_t* b_empty = b_full + kStagesB;
+  uint64_t* acc_full = b_empty + kStagesB;  // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2] (the leader's counts both CTAs' epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* cnt = const_cast<int*>(abort_flag + 1);  // [E]
+  int* prefix = cnt + 1024;                     // [E + 1]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cta_rank_in_cluster();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x) >> 1;
+  const int npairs = static_cast<int>(gridDim.x) >> 1;
+  const int E = args.E;
+  // weight blocks per expert: up = 256 rows of gate and of up; down = 512 rows
+  const int W = kUp ? args.rows_per_expert / (2 * kBM) : args.rows_per_expert / (4 * kBM);
+
+  for (int e = tid; e < E; e += kThreads) cnt[e] = args.expert_counts[e];
+  if (tid == 0) *abort_flag = 0;
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int lo = min(E, lane * per), hi = min(E, lo + per);
+    int sum = 0;
+    for (int e = lo; e < hi; ++e) sum += W * ((cnt[e] + kNmax - 1) / kNmax);
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+    for (int e = lo; e < hi; ++e) {
+      prefix[e] = run;
+      run += W * ((cnt[e] + kNmax - 1) / kNmax);
+    }
+    if (lane == 31) prefix[E] = incl;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStagesA; ++s) {
+      mbar_init(&a_full[s], 1);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesB; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int total = prefix[E];
+  // Both CTAs of a pair see the same tile count, so they leave together.
+  if (pair >= total) return;
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before_sync();
+  cluster_sync_all();  // the peer's barriers are initialised and both CTAs hold tensor memory
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = args.kdim / kBK;
+  const int nslots = args.M * args.top_k;
+
+  if (warp == 0) {
+    // ------------------------------------------------ weight producer (both CTAs)
+    if (lane == 0) {
+      prefetch_tensor_map(&tm_a0);
+      if (kUp) prefetch_tensor_map(&tm_a1);
+    }
+    int ka = 0;
+    bool alive = true;
+    for (int tile = pair; tile < total && alive; tile += npairs) {
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
+      const bool single_use = cnt[c.e] <= kNmax;
+      const uint64_t pol = single_use ? l2_policy_evict_first() : l2_policy_evict_normal();
+      const int base = c.e * args.rows_per_expert + static_cast<int>(rank) * kBM;
+      const int row_a0 = kUp ? base + c.w * 2 * kBM : base + c.w * 4 * kBM;
+      const int row_a1 = kUp ? row_a0 : row_a0 + 2 * kBM;
+      for (int k = 0; k < nk; ++k, ++ka) {
+        const int s = ka % kStagesA;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&a_empty[s], ((ka / kStagesA) & 1) ^ 1, abort_flag);
+          if (ok && leader) mbar_arrive_expect_tx(&a_full[s], 2 * C::kAStage);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            set_error(args.err, kErrTimeout);
+          }
+          alive = false;
+          break;
+        }
+        uint8_t* st = a_ring + s * C::kAStage;
+        const uint32_t bar = cluster_addr(&a_full[s], 0);
+        if (lane == 0)
+          tma_load_2d_pair(&tm_a0, bar, st, k * kBK, row_a0, pol);
+        else if (lane == 1)
+          tma_load_2d_pair(kUp ? &tm_a1 : &tm_a0, bar, st + kBoxBytes, k * kBK, row_a1, pol);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------ token-row producer (both CTAs)
+    if (lane == 0) prefetch_tensor_map(&tm_b);
+    const uint64_t pol_b = l2_policy_evict_normal();
+    int kb = 0;
+    bool alive = true;
+    for (int tile = pair; tile < total && alive; tile += npairs) {
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
+      const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
+      const int N = (nrows + 15) & ~15;
+      const int half = N / 2;
+      const int row0 = args.expert_offsets[c.e] + c.t * kNmax + static_cast<int>(rank) * half;
+      const int nbox = (half + kBRows - 1) / kBRows;
+      for (int k = 0; k < nk; ++k, ++kb) {
+        const int s = kb % kStagesB;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&b_empty[s], ((kb / kStagesB) & 1) ^ 1, abort_flag);
+          if (ok && leader) mbar_arrive_expect_tx(&b_full[s], 2 * nbox * kBRows * kBK * 2);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            set_error(args.err, kErrTimeout);
+          }
+          alive = false;
+          break;
+        }
+        uint8_t* st = b_ring + s * C::kBStage;
+        if (lane < nbox)
+          tma_load_2d_pair(&tm_b, cluster_addr(&b_full[s], 0), st + lane * kBRows * kBK * 2, k * kBK,
+                           row0 + lane * kBRows, pol_b);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader only)
+    if (leader && lane == 0) {
+      int ka = 0, kb = 0, j = 0;
+      bool alive = true;
+      for (int tile = pair; tile < total && alive; tile += npairs, ++j) {
+        const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
+        const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
+        const int N = (nrows + 15) & ~15;
+        const uint32_t idesc = umma_idesc_bf16(2 * kBM, N);
+        const int buf = j % C::kAccBufs;
+        const int use = j / C::kAccBufs;
+        if (!mbar_wait_bounded(&acc_empty[buf], (use & 1) ^ 1, abort_flag)) {
+          *abort_flag = 1;
+          set_error(args.err, kErrTimeout);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d0 = tmem + buf * C::kAccCols;
+        const uint32_t d1 = d0 + kNmax;
+        for (int k = 0; k < nk; ++k, ++ka, ++kb) {
+          const int sa = ka % kStagesA, sb = kb % kStagesB;
+          if (!mbar_wait_bounded(&a_full[sa], (ka / kStagesA) & 1, abort_flag) ||
+              !mbar_wait_bounded(&b_full[sb], (kb / kStagesB) & 1, abort_flag)) {
+            *abort_flag = 1;
+            set_error(args.err, kErrTimeout);
+            alive = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint64_t da0 = umma_desc_sw128(a_ring + sa * C::kAStage);
+          const uint64_t da1 = umma_desc_sw128(a_ring + sa * C::kAStage + kBoxBytes);
+          const uint64_t db = umma_desc_sw128(b_ring + sb * C::kBStage);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t acc = (k | kk) != 0 ? 1u : 0u;
+            umma_bf16_pair(d0, da0 + 2 * kk, db + 2 * kk, idesc, acc);
+            umma_bf16_pair(d1, da1 + 2 * kk, db + 2 * kk, idesc, acc);
+          }
+          umma_commit_pair(&a_empty[sa]);
+          umma_commit_pair(&b_empty[sb]);
+        }
+        umma_commit_pair(&acc_full[buf]);  // also on an abort, so neither epilogue is left waiting
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------ epilogue (both CTAs: their own 128 rows)
+    const int q = warp & 3;
+    const int half_c = (warp - 4) >> 2;
+    int j = 0;
+    for (int tile = pair; tile < total; tile += npairs, ++j) {
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
+      const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
+      const int N = (nrows + 15) & ~15;
+      const int row0 = args.expert_offsets[c.e] + c.t * kNmax;
+      const int buf = j % C::kAccBufs;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(&acc_full[buf], (j / C::kAccBufs) & 1, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      tc_fence_after_sync();
+      const bool go = __shfl_sync(0xffffffffu, ok && !*abort_flag, 0);
+      if (!go) {
+        if (lane == 0 && !ok) set_error(args.err, kErrTimeout);
+        break;
+      }
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
+      int ids[kNmax / 32];
+      if (!kUp) {
+#pragma unroll
+        for (int i = 0; i < kNmax / 32; ++i) {
+          const int n = lane + 32 * i;
+          ids[i] = (n < nrows) ? args.sorted_ids[row0 + n] : -1;
+        }
+      }
+      auto* out = reinterpret_cast<__nv_bfloat16*>(args.out);
+      const int colbase = kUp ? c.w * 2 * kBM + static_cast<int>(rank) * kBM
+                              : c.w * 4 * kBM + static_cast<int>(rank) * kBM;
+      for (int cb = 16 * half_c; cb < N; cb += 32) {
+        uint32_t v0[16], v1[16];
+        tmem_load_16(lane_base + cb, v0);
+        tmem_load_16(lane_base + kNmax + cb, v1);
+        tmem_load_wait();
+        const int id_word = kUp ? 0 : pick<kNmax / 32>(ids, cb >> 5);
+#pragma unroll
+        for (int qq = 0; qq < 16; ++qq) {
+          const int n = cb + qq;
+          const int col = colbase + q * 32 + lane;
+          if (kUp) {
+            if (n < nrows) {
+              const float g = __uint_as_float(v0[qq]);
+              const float u = __uint_as_float(v1[qq]);
+              out[static_cast<size_t>(row0 + n) * args.out_ld + col] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+            }
+          } else {
+            const int id = __shfl_sync(0xffffffffu, id_word, (cb & 31) + qq);
+            if (n < nrows && id >= 0 && id < nslots) {
+              out[static_cast<size_t>(id) * args.out_ld + col] = __float2bfloat16_rn(__uint_as_float(v0[qq]));
+              out[static_cast<size_t>(id) * args.out_ld + col + 2 * kBM] =
+                  __float2bfloat16_rn(__uint_as_float(v1[qq]));
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[buf], 0));
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the other may still use its shared or tensor memory
+  if (warp == 1) tmem_dealloc_pair(tmem, 512);
+}
+
+template <bool kUp, int kNmax, int kStagesA, int kStagesB>
+cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const GroupedGemmArgs& args,
+                        int num_sms, cudaStream_t stream) {
+  using C = QCfg<kNmax, kStagesA, kStagesB>;
+  auto kern = pair_gemm_kernel<kUp, kNmax, kStagesA, kStagesB>;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  static bool done[64] = {};
+  if (dev < 64 && !done[dev]) {
+    st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (st != cudaSuccess) return st;
+    done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, args);
+}
+
+}  // namespace
+
+cudaError_t launch_pair_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                           const GroupedGemmArgs& args, int nmax, int num_sms, cudaStream_t stream) {
+  if (args.rows_per_expert % (2 * kBM) != 0) return cudaErrorInvalidValue;
+  if (nmax >= 256) return launch_pair<true, 256, 5, 3>(w_gate, w_up, x_rows, args, num_sms, stream);
+  return launch_pair<true, 128, 5, 6>(w_gate, w_up, x_rows, args, num_sms, stream);
+}
+
+cudaError_t launch_pair_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
+                             int nmax, int num_sms, cudaStream_t stream) {
+  if (args.rows_per_expert % (4 * kBM) != 0) return cudaErrorInvalidValue;
+  if (nmax >= 256) return launch_pair<false, 256, 5, 3>(w_down, w_down, h_rows, args, num_sms, stream);
+  return launch_pair<false, 128, 5, 6>(w_down, w_down, h_rows, args, num_sms, stream);
+}
+
+}  // namespace moe

@@ -72,6 +72,14 @@ cudaError_t launch_grouped_up(const CUtensorMap& w_gate, const CUtensorMap& w_up
 // xg[r] = x[sorted_ids[r] / top_k] for the real plan rows r < ntpp.
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* sorted_ids, const int32_t* ntpp, int M, int top_k,
                                int H, int cap, uint16_t* xg, cudaStream_t stream);
+// 2-SM pair variants of the persistent kernels (gemm_pair.cu): token tiles of
+// `nmax` plan rows (128 or 256) split over the two CTAs of a cluster; the
+// token-row tensor is plan-ordered (x gathered, or h) in 32-row boxes.
+cudaError_t launch_pair_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
+                           const GroupedGemmArgs& args, int nmax, int num_sms, cudaStream_t stream);
+cudaError_t launch_pair_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
+                             int nmax, int num_sms, cudaStream_t stream);
+
 // Decode up projection that builds the plan itself from topk_ids (32-row
 // token tiles, x rows gathered by token id) and writes it for the down and
 // finalize kernels: the align step folded into the up kernel.

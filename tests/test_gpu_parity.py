@@ -240,6 +240,7 @@ def test_grouped_up_down(case, nmax, gather, persistent, deep_b, monkeypatch):
     monkeypatch.setenv("MOE_GEMM_NMAX", nmax)
     monkeypatch.setenv("MOE_UP_GATHER", gather)
     monkeypatch.setenv("MOE_GEMM_PERSISTENT", persistent)
+    monkeypatch.setenv("MOE_GEMM_PAIR", "0")  # the single-SM kernels (pairs: test_gpu_pair.py)
     cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + case["E"], **case)
     d = to_dev(cfg)
     hb = host_bits(d)
