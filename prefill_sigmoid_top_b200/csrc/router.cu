@@ -13,8 +13,9 @@
 //     partial l of each of the warp's (token, expert) pairs; x and w_router
 //     arrive through a shared-memory ring of 256-element slabs (cp.async).
 //     Few tokens: 8 tokens x 1 expert per warp, 16 slabs in flight.  Many
-//     tokens: 8 tokens x 8 experts per warp, the fmas of token pairs issued
-//     as paired fp32 fmas.
+//     tokens: 8 tokens x 8 experts per warp.  Every fma takes its bf16
+//     operands directly (fma.rn.f32.bf16: exact product, one rounding), so no
+//     bf16 -> fp32 conversion is issued.
 //  2. router_topk_kernel: one warp per token selects the K largest logits
 //     (descending; equal logits -> lower expert id) by K rounds of a warp
 //     argmax, then w_k = s_k / sum s with s = 1 / (1 + exp(-z)).
@@ -30,11 +31,6 @@
 
 namespace moe {
 namespace {
-
-__device__ __forceinline__ float elem(const uint4& v, int i) {
-  const uint32_t w = (i < 2) ? v.x : (i < 4) ? v.y : (i < 6) ? v.z : v.w;
-  return (i & 1) ? bf16_hi(w) : bf16_lo(w);
-}
 
 // ---------------------------------------------------------------------------
 // Logits.  x and w_router reach the warps through a ring of kStages slabs of
@@ -68,23 +64,31 @@ struct StagedCfg {
   static_assert(kTt * kTe <= 64, "pairs per warp");
 };
 
-// Two fp32 fmas in one instruction (each lane of the pair is an ordinary
-// round-to-nearest fma): d.{lo,hi} = a.{lo,hi} * b.{lo,hi} + d.{lo,hi}.
-__device__ __forceinline__ void fma2(uint64_t& d, uint64_t a, uint64_t b) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
-}
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 unpack2(uint64_t v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
+// fp32 fma with bf16 multiplicands: c + a*b rounded once, a and b taken
+// exactly (a product of two bf16 values is exact in fp32), so the result is
+// the same as fmaf(float(a), float(b), c) without the two conversions.
+// kHi selects the high or the low bf16 half of each 32-bit word.
+template <bool kHi>
+__device__ __forceinline__ float fma_bf16(uint32_t aw, uint32_t bw, float c) {
+  float d = c;
+  if (kHi)
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "+f"(d)
+        : "r"(aw), "r"(bw));
+  else
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t}"
+        : "+f"(d)
+        : "r"(aw), "r"(bw));
+  return d;
 }
 
-template <int kTt, int kTe, int kWt, int kWe, int kStages, bool kPair>
+__device__ __forceinline__ uint32_t word(const uint4& v, int w) {
+  return w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+}
+
+template <int kTt, int kTe, int kWt, int kWe, int kStages>
 __global__ void __launch_bounds__(kWt * kWe * 32) router_logits_staged_kernel(const uint16_t* __restrict__ x,
                                                                              const uint16_t* __restrict__ w_router,
                                                                              const float* __restrict__ bias, int M,
@@ -116,19 +120,11 @@ __global__ void __launch_bounds__(kWt * kWe * 32) router_logits_staged_kernel(co
     }
   };
 
-  // kPair: the accumulators of tokens 2u and 2u+1 (same expert) share one
-  // 64-bit register and advance together in one paired fma.
-  static_assert(!kPair || kTt % 2 == 0, "token pairs");
   float acc[kTt][kTe];
-  uint64_t acc2[kTt / 2][kTe];
 #pragma unroll
   for (int t = 0; t < kTt; ++t)
 #pragma unroll
     for (int q = 0; q < kTe; ++q) acc[t][q] = 0.0f;
-#pragma unroll
-  for (int u = 0; u < kTt / 2; ++u)
-#pragma unroll
-    for (int q = 0; q < kTe; ++q) acc2[u][q] = 0ull;
 
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
@@ -148,43 +144,16 @@ __global__ void __launch_bounds__(kWt * kWe * 32) router_logits_staged_kernel(co
 #pragma unroll
     for (int q = 0; q < kTe; ++q)
       wv[q] = *reinterpret_cast<const uint4*>(st + (C::kRowsX + we * kTe + q) * 512 + lane * 16);
-    if (kPair) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {  // increasing h inside the chunk
-        uint64_t xp[kTt / 2], wp[kTe];
+    for (int i = 0; i < 8; ++i)  // increasing h inside the chunk
 #pragma unroll
-        for (int u = 0; u < kTt / 2; ++u) xp[u] = pack2(elem(xv[2 * u], i), elem(xv[2 * u + 1], i));
+      for (int t = 0; t < kTt; ++t)
 #pragma unroll
-        for (int q = 0; q < kTe; ++q) {
-          const float w = elem(wv[q], i);
-          wp[q] = pack2(w, w);
-        }
-#pragma unroll
-        for (int u = 0; u < kTt / 2; ++u)
-#pragma unroll
-          for (int q = 0; q < kTe; ++q) fma2(acc2[u][q], xp[u], wp[q]);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)  // increasing h inside the chunk
-#pragma unroll
-        for (int t = 0; t < kTt; ++t)
-#pragma unroll
-          for (int q = 0; q < kTe; ++q) acc[t][q] = __fmaf_rn(elem(xv[t], i), elem(wv[q], i), acc[t][q]);
-    }
+        for (int q = 0; q < kTe; ++q)
+          acc[t][q] = (i & 1) ? fma_bf16<true>(word(xv[t], i >> 1), word(wv[q], i >> 1), acc[t][q])
+                              : fma_bf16<false>(word(xv[t], i >> 1), word(wv[q], i >> 1), acc[t][q]);
     __syncthreads();  // the stage may be refilled
   }
-  if (kPair) {
-#pragma unroll
-    for (int u = 0; u < kTt / 2; ++u)
-#pragma unroll
-      for (int q = 0; q < kTe; ++q) {
-        const float2 v = unpack2(acc2[u][q]);
-        acc[2 * u][q] = v.x;
-        acc[2 * u + 1][q] = v.y;
-      }
-  }
-
 #pragma unroll
   for (int t = 0; t < kTt; ++t)
 #pragma unroll
@@ -200,11 +169,11 @@ __global__ void __launch_bounds__(kWt * kWe * 32) router_logits_staged_kernel(co
     }
 }
 
-template <int kTt, int kTe, int kWt, int kWe, int kStages, bool kPair>
+template <int kTt, int kTe, int kWt, int kWe, int kStages>
 cudaError_t launch_staged(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
                           float* logits, cudaStream_t stream) {
   using C = StagedCfg<kTt, kTe, kWt, kWe, kStages>;
-  auto kern = router_logits_staged_kernel<kTt, kTe, kWt, kWe, kStages, kPair>;
+  auto kern = router_logits_staged_kernel<kTt, kTe, kWt, kWe, kStages>;
   int dev = 0;
   cudaError_t st = cudaGetDevice(&dev);
   if (st != cudaSuccess) return st;
@@ -355,8 +324,8 @@ __global__ void __launch_bounds__(128) router_topk_ext_kernel(const float* __res
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
                                  float* logits, cudaStream_t stream) {
   if (M <= 64)  // few tokens: one expert per warp, so that many warps share the reads of w_router; deep ring
-    return launch_staged<8, 1, 1, 4, 16, false>(x, w_router, bias, M, H, E, logits, stream);
-  return launch_staged<8, 8, 2, 2, 4, true>(x, w_router, bias, M, H, E, logits, stream);
+    return launch_staged<8, 1, 1, 4, 16>(x, w_router, bias, M, H, E, logits, stream);
+  return launch_staged<8, 8, 2, 2, 4>(x, w_router, bias, M, H, E, logits, stream);
 }
 
 cudaError_t launch_router_topk(const float* logits, int M, int E, int K, int32_t* topk_ids, float* topk_w,
