@@ -107,7 +107,9 @@ class ClockSampler:
         self.period = period_s
         self.samples = []
         self.max_mhz = None
+        self.error = None
         self._stop = threading.Event()
+        self._ready = threading.Event()
         self._thread = None
 
     def _handle(self, nv):
@@ -126,17 +128,22 @@ class ClockSampler:
             self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
             get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
                 nv.nvmlDeviceGetCurrentClocksThrottleReasons
-            while not self._stop.is_set():
+            while True:
                 self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(get_reasons(h))))
+                self._ready.set()
+                if self._stop.is_set():
+                    break
                 time.sleep(self.period)
             nv.nvmlShutdown()
         except Exception as e:  # no NVML: report no clock record rather than fail the bench
             self.error = repr(e)
+        finally:
+            self._ready.set()
 
     def __enter__(self):
         self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
-        time.sleep(0.01)
+        self._ready.wait(timeout=5.0)  # the timed region starts once sampling has begun
         return self
 
     def __exit__(self, *exc):
@@ -145,7 +152,7 @@ class ClockSampler:
 
     def summary(self):
         if not self.samples:
-            return None
+            return None if self.error is None else {"error": self.error}
         reasons = set()
         for _, r in self.samples:
             for bit, name in self.REASONS.items():

@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(
 // `blockIdx.x`, row r <- token sorted_ids[row0 + r] / top_k.  The tile's token
 // ids are staged in shared memory first; then every thread copies independent
 // 16-byte code chunks and 4-byte scale words (four column blocks of one scale
-// atom row), so many loads are in flight.  Rows past the expert's count are
+// atom row), so many loads are in flight; blockIdx.y splits the columns over
+// 8 CTAs per tile, so that each thread has few copies to chain.  Rows past the expert's count are
 // not written (as above).
 __global__ void __launch_bounds__(256) gather_tiles_kernel(
     const uint8_t* __restrict__ tok_codes, const uint8_t* __restrict__ tok_scales,
@@ -275,18 +276,22 @@ __global__ void __launch_bounds__(256) gather_tiles_kernel(
   __syncthreads();
   const int cb16 = cols / 32;  // 16-byte code chunks per row
   const int nw = cols / 64;    // scale words per row
+  // this CTA's slice of the chunks [c0, c0 + cw) and scale words [a0, a0 + aw)
+  const int cper = (cb16 + gridDim.y - 1) / gridDim.y, aper = (nw + gridDim.y - 1) / gridDim.y;
+  const int c0 = blockIdx.y * cper, cw = max(0, min(cb16, c0 + cper) - c0);
+  const int a0 = blockIdx.y * aper, aw = max(0, min(nw, a0 + aper) - a0);
   const uint4* src = reinterpret_cast<const uint4*>(tok_codes);
   uint4* dst = reinterpret_cast<uint4*>(codes) + static_cast<int64_t>(ti) * 128 * cb16;
 #pragma unroll 4
-  for (int i = tid; i < nrows * cb16; i += blockDim.x) {
-    const int r = i / cb16, c = i - r * cb16;
+  for (int i = tid; i < nrows * cw; i += blockDim.x) {
+    const int r = i / cw, c = c0 + (i - r * cw);
     const int t = s_tok[r];
     dst[static_cast<int64_t>(r) * cb16 + c] = t >= 0 ? src[static_cast<int64_t>(t) * cb16 + c] : make_uint4(0, 0, 0, 0);
   }
   const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(tok_scales);
 #pragma unroll 4
-  for (int i = tid; i < nrows * nw; i += blockDim.x) {
-    const int r = i / nw, a = i - r * nw;
+  for (int i = tid; i < nrows * aw; i += blockDim.x) {
+    const int r = i / aw, a = a0 + (i - r * aw);
     const int t = s_tok[r];
     *reinterpret_cast<uint32_t*>(atoms + (static_cast<int64_t>(ti) * nw + a) * 512 + (r % 32) * 16 + (r / 32) * 4) =
         t >= 0 ? ssrc[static_cast<int64_t>(t) * nw + a] : 0u;
@@ -718,7 +723,7 @@ cudaError_t launch_amax_plan_rows(const uint16_t* h, const int32_t* sorted_ids, 
 cudaError_t launch_quantize_tiles(const uint16_t* src, const int32_t* counts, const int32_t* offsets, int E, int cols,
                                   int tiles_ub, const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms,
                                   cudaStream_t stream) {
-  const int slices = std::max(1, cols / 16 / 64);  // 64 column blocks (1024 elements) per CTA
+  const int slices = std::max(1, cols / 16 / 16);  // 16 column blocks (256 elements) per CTA
   quantize_tiles_kernel<<<dim3(tiles_ub, slices), 256, 0, stream>>>(src, counts, offsets, E, cols, amax_bits, codes,
                                                                     atoms);
   return cudaGetLastError();
@@ -736,7 +741,7 @@ cudaError_t launch_quantize_rows(const uint16_t* src, int64_t rows, int64_t cols
 cudaError_t launch_gather_tiles(const uint8_t* tok_codes, const uint8_t* tok_scales, const int32_t* sorted_ids,
                                 const int32_t* counts, const int32_t* offsets, int E, int top_k, int nslots, int cols,
                                 int tiles_ub, uint8_t* codes, uint8_t* atoms, cudaStream_t stream) {
-  gather_tiles_kernel<<<tiles_ub, 256, 0, stream>>>(tok_codes, tok_scales, sorted_ids, counts, offsets, E, top_k,
+  gather_tiles_kernel<<<dim3(tiles_ub, 8), 256, 0, stream>>>(tok_codes, tok_scales, sorted_ids, counts, offsets, E, top_k,
                                                     nslots, cols, codes, atoms);
   return cudaGetLastError();
 }
