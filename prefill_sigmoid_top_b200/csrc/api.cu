@@ -83,12 +83,14 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
-// Token-tile width of the grouped kernels, from the mean routed rows per
-// expert (known on the host without reading the plan back): decode shapes
-// (<= 24) use 32-row tiles, larger ones 128-row tiles.  256-row tiles measured
-// slower on the batch and prefill workloads (one accumulator set fills tensor
-// memory), so they run only when asked for.  MOE_GEMM_NMAX=32|128|256
-// overrides (the tests cover every variant).
+// Token-tile width of the single-SM grouped kernels, from the mean routed rows
+// per expert (known on the host without reading the plan back): decode shapes
+// (<= 24) use 32-row tiles, larger ones 128-row tiles (which also selects the
+// persistent path; there the 2-SM pair kernels pick their own width, see
+// pair_nmax).  Single-SM 256-row tiles measured slower on the batch and
+// prefill workloads (one accumulator set fills tensor memory), so they run
+// only when asked for.  MOE_GEMM_NMAX=32|128|256 overrides (the tests cover
+// every variant).
 int choose_nmax(const moe_shape_t& s) {
   if (const char* env = std::getenv("MOE_GEMM_NMAX")) {
     const int v = std::atoi(env);
@@ -154,10 +156,12 @@ size_t blob_codes_bytes(const moe_shape_t& s, int which) {
   return static_cast<size_t>(r) * c / 2;
 }
 
-// Whether the batch/prefill shapes run the persistent kernel (one CTA per SM,
-// deep weight ring, double-buffered accumulators).  MOE_GEMM_PERSISTENT=0|1
-// overrides; the up projection also needs the plan-ordered copy of x, so it
-// only takes this path when the caller provides that workspace.
+// Whether the batch/prefill shapes take the persistent path (one CTA or one
+// 2-SM pair per SM pair, deep weight ring): the pair kernels by default, the
+// single-SM persistent kernels for shapes the pairs do not take or with
+// MOE_GEMM_PAIR=0.  MOE_GEMM_PERSISTENT=0|1 overrides; the up projection also
+// needs the plan-ordered copy of x, so it only takes this path when the
+// caller provides that workspace.
 bool want_persistent(const moe_shape_t& s) {
   if (const char* env = std::getenv("MOE_GEMM_PERSISTENT")) {
     if (std::strcmp(env, "0") == 0) return false;
