@@ -156,8 +156,8 @@ size_t blob_codes_bytes(const moe_shape_t& s, int which) {
   return static_cast<size_t>(r) * c / 2;
 }
 
-// Whether the batch/prefill shapes take the persistent path (one CTA or one
-// 2-SM pair per SM pair, deep weight ring): the pair kernels by default, the
+// Whether the batch/prefill shapes take the persistent path (one CTA per SM,
+// or one cluster per two SMs; deep weight ring): the pair kernels by default, the
 // single-SM persistent kernels for shapes the pairs do not take or with
 // MOE_GEMM_PAIR=0.  MOE_GEMM_PERSISTENT=0|1 overrides; the up projection also
 // needs the plan-ordered copy of x, so it only takes this path when the
