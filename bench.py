@@ -29,8 +29,9 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 # ncu DRAM traffic of the dominant kernel, per launch, measured on the decode
-# workload (profiles/grouped_up_decode_m8_E32.md).  Valid only while the kernel
-# sources hash to KERNEL_HASH; otherwise "traffic" is reported as null.
+# workload (a capture on its E=32 copy, scaled by the touched experts).  Valid
+# only while the kernel sources hash to the recorded value; otherwise "traffic"
+# is reported as null.
 NCU_TRAFFIC = {
     # decode M=8: E=32 capture (1.8243 GB for 31 touched experts) scaled to 95 touched experts
     1: (5_590_700_000, "bf42fabd738f6afa"),
@@ -63,7 +64,7 @@ def parse_args(argv=None):
 
 def workload(args):
     from prefill_sigmoid_top_b200 import inputs
-    cfg = inputs.CONFIGS[args.config]
+    cfg = inputs.WORKLOADS[args.config]
     if args.experts:
         cfg = cfg.with_(E=args.experts, name=f"{cfg.name}_E{args.experts}")
     if args.tokens:

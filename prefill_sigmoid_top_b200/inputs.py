@@ -67,7 +67,7 @@ class MoEConfig:
         return replace(self, **kw)
 
 
-CONFIGS = {
+WORKLOADS = {
     0: MoEConfig("tiny", M=16, H=256, I=128, E=8, K=2, B=16, seed=0, bias="zero"),
     1: MoEConfig("decode_m8", M=8, H=7168, I=2048, E=256, K=16, B=16, seed=1),
     2: MoEConfig("batch_m512", M=512, H=7168, I=2048, E=256, K=16, B=64, seed=2),

@@ -35,7 +35,7 @@ def ratio_for(tree, bias, K, E):
 
 
 def main():
-    cfg = inputs.CONFIGS[3]
+    cfg = inputs.WORKLOADS[3]
     w_router, _, _, x = inputs.router_inputs(cfg, alpha=1.0)
     tree = oracle.router_logits(bf16_bits(x), bf16_bits(w_router), None)  # bias-free canonical sums
     lo, hi = 0.0, 2.0

@@ -57,7 +57,7 @@ def test_quantize_bitexact_against_oracle():
 
 
 def test_quantize_bitexact_expert_weights():
-    cfg = inputs.CONFIGS[0].with_(E=4, I=256, H=512, seed=17)
+    cfg = inputs.WORKLOADS[0].with_(E=4, I=256, H=512, seed=17)
     wg, _, wd = inputs.expert_weights(cfg, DEV)
     for w in (wg, wd):
         codes, scales, gs = moe.quantize_nvfp4(w)
@@ -100,7 +100,7 @@ NVFP4_CASES = [dict(M=40, H=512, I=256, E=16, K=4, B=16), dict(M=300, H=256, I=5
 
 @pytest.mark.parametrize("case", NVFP4_CASES, ids=lambda c: f"M{c['M']}_E{c['E']}")
 def test_nvfp4_grouped_and_layer(case):
-    cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + 5, **case)
+    cfg = inputs.WORKLOADS[0].with_(bias="normal", seed=case["M"] + 5, **case)
     d = inputs.make_inputs(cfg, DEV)
     shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
     nw = moe.nvfp4_weights(d["w_gate"], d["w_up"], d["w_down"], shape)
@@ -154,7 +154,7 @@ def test_nvfp4_rejects_unsupported_intermediate():
 
 @pytest.mark.slow
 def test_nvfp4_layer_full_size_sampled():
-    cfg = inputs.CONFIGS[4]
+    cfg = inputs.WORKLOADS[4]
     d = inputs.make_inputs(cfg, DEV)
     shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
     nw = moe.nvfp4_weights(d["w_gate"], d["w_up"], d["w_down"], shape)

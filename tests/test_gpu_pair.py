@@ -32,7 +32,7 @@ def test_pair_up_down(case, pair, monkeypatch):
     monkeypatch.setenv("MOE_UP_GATHER", "pregather")
     monkeypatch.setenv("MOE_GEMM_NMAX", "128")
     monkeypatch.setenv("MOE_GEMM_PAIR", pair)
-    cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + 7 * case["E"], **case)
+    cfg = inputs.WORKLOADS[0].with_(bias="normal", seed=case["M"] + 7 * case["E"], **case)
     d = to_dev(cfg)
     hb = host_bits(d)
     ids_o, _ = oracle.route(hb["x"], hb["w_router"], hb["bias"], cfg.K)

@@ -72,7 +72,7 @@ SMALL_ROUTER_SHAPES = [
 
 @pytest.mark.parametrize("M,H,E,K,bias", SMALL_ROUTER_SHAPES)
 def test_router_bitexact_small(M, H, E, K, bias):
-    cfg = inputs.CONFIGS[0].with_(M=M, H=H, E=E, K=K, bias=bias, seed=M * 7 + E)
+    cfg = inputs.WORKLOADS[0].with_(M=M, H=H, E=E, K=K, bias=bias, seed=M * 7 + E)
     w_r, b, g, x = inputs.router_inputs(cfg)
     ids, w = moe.route(x.to(DEV), w_r.to(DEV), b.to(DEV), K)
     ids_o, w_o = oracle.route(bf16_bits(x), bf16_bits(w_r), b.numpy(), K)
@@ -92,7 +92,7 @@ def test_router_ties_exact():
 
 @pytest.mark.parametrize("cid", [1, 2, 3, 4])
 def test_router_bitexact_full_size(cid):
-    cfg = inputs.CONFIGS[cid]
+    cfg = inputs.WORKLOADS[cid]
     w_r, b, g, x = inputs.router_inputs(cfg)
     ids, w = moe.route(x.to(DEV), w_r.to(DEV), b.to(DEV), cfg.K)
     ids_o, w_o = oracle.route(bf16_bits(x), bf16_bits(w_r), b.numpy(), cfg.K)
@@ -241,7 +241,7 @@ def test_grouped_up_down(case, nmax, gather, persistent, deep_b, monkeypatch):
     monkeypatch.setenv("MOE_UP_GATHER", gather)
     monkeypatch.setenv("MOE_GEMM_PERSISTENT", persistent)
     monkeypatch.setenv("MOE_GEMM_PAIR", "0")  # the single-SM kernels (pairs: test_gpu_pair.py)
-    cfg = inputs.CONFIGS[0].with_(bias="normal", seed=case["M"] + case["E"], **case)
+    cfg = inputs.WORKLOADS[0].with_(bias="normal", seed=case["M"] + case["E"], **case)
     d = to_dev(cfg)
     hb = host_bits(d)
     ids_o, w_o = oracle.route(hb["x"], hb["w_router"], hb["bias"], cfg.K)
@@ -307,10 +307,10 @@ def run_layer(d, cfg, stream_sync=True):
 
 
 LAYER_SMALL = [
-    inputs.CONFIGS[0],
-    inputs.CONFIGS[0].with_(M=40, H=512, I=256, E=16, K=4, B=16, seed=11, bias="normal"),
-    inputs.CONFIGS[0].with_(M=257, H=768, I=256, E=32, K=8, B=64, seed=12, bias="zipf"),
-    inputs.CONFIGS[0].with_(M=3, H=256, I=128, E=4, K=4, B=16, seed=13, bias="normal"),
+    inputs.WORKLOADS[0],
+    inputs.WORKLOADS[0].with_(M=40, H=512, I=256, E=16, K=4, B=16, seed=11, bias="normal"),
+    inputs.WORKLOADS[0].with_(M=257, H=768, I=256, E=32, K=8, B=64, seed=12, bias="zipf"),
+    inputs.WORKLOADS[0].with_(M=3, H=256, I=128, E=4, K=4, B=16, seed=13, bias="normal"),
 ]
 
 
@@ -344,7 +344,7 @@ def _sample_tokens(ids_o, n_random, seed):
 @pytest.mark.slow
 @pytest.mark.parametrize("cid", [1, 2, 3])
 def test_layer_full_size_sampled(cid):
-    cfg = inputs.CONFIGS[cid]
+    cfg = inputs.WORKLOADS[cid]
     d = to_dev(cfg)
     g = run_layer(d, cfg)
     hb = host_bits(d)

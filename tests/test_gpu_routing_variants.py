@@ -44,27 +44,27 @@ def _run(cfg, variant, bias_override=None):
 @pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("M,E,K", [(37, 64, 6), (19, 256, 16), (9, 1024, 8)])
 def test_variants_small(variant, M, E, K):
-    cfg = inputs.CONFIGS[0].with_(M=M, H=512, E=E, K=K, bias="normal", seed=M + E)
+    cfg = inputs.WORKLOADS[0].with_(M=M, H=512, E=E, K=K, bias="normal", seed=M + E)
     _run(cfg, variant)
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
 def test_selection_only_bias_changes_picks(variant):
     # a strong ramp bias: picks follow the key, weights follow the unbiased logit
-    cfg = inputs.CONFIGS[0].with_(M=33, H=256, E=64, K=8, seed=5)
+    cfg = inputs.WORKLOADS[0].with_(M=33, H=256, E=64, K=8, seed=5)
     ramp = torch.from_numpy((np.arange(cfg.E, dtype=np.float32) - cfg.E / 2) * 0.2)
     _run(cfg, variant, bias_override=ramp)
 
 
 @pytest.mark.parametrize("cid", [1, 3])
 def test_variants_full_size(cid):
-    cfg = inputs.CONFIGS[cid]
+    cfg = inputs.WORKLOADS[cid]
     _run(cfg, (moe.SCORE_SOFTMAX, True, 2.5, True))
     _run(cfg, (moe.SCORE_SIGMOID, False, 1.0, False))
 
 
 def test_default_options_equal_route_bitwise():
-    cfg = inputs.CONFIGS[2]
+    cfg = inputs.WORKLOADS[2]
     w_r, b, g, x = inputs.router_inputs(cfg)
     xd, wd, bd = x.to(DEV), w_r.to(DEV), b.to(DEV)
     ids0, w0 = moe.route(xd, wd, bd, cfg.K)

@@ -43,7 +43,7 @@ def _plan_np(p):
 
 @pytest.mark.parametrize("M,H,I,E,K,B", CASES)
 def test_routed_up_matches_align_plus_up(M, H, I, E, K, B):
-    cfg = inputs.CONFIGS[0].with_(M=M, H=H, I=I, E=E, K=K, B=B, bias="normal", seed=M * 3 + E)
+    cfg = inputs.WORKLOADS[0].with_(M=M, H=H, I=I, E=E, K=K, B=B, bias="normal", seed=M * 3 + E)
     d = _weights(cfg)
     shape = moe.Shape(M, H, I, E, K, B)
     ids, _ = moe.route(d["x"], d["w_router"], d["bias"], K)
@@ -68,7 +68,7 @@ def test_routed_up_matches_align_plus_up(M, H, I, E, K, B):
 
 def test_routed_up_flags_invalid_ids():
     M, H, I, E, K, B = 16, 256, 128, 8, 2, 16
-    cfg = inputs.CONFIGS[0].with_(M=M, H=H, I=I, E=E, K=K, B=B, seed=3)
+    cfg = inputs.WORKLOADS[0].with_(M=M, H=H, I=I, E=E, K=K, B=B, seed=3)
     d = _weights(cfg)
     ids = torch.randint(0, E, (M, K), dtype=torch.int32, device=DEV)
     ids[3, 1] = E        # out of range: flagged on the device, never read as an expert
@@ -81,7 +81,7 @@ def test_routed_up_flags_invalid_ids():
 
 @pytest.mark.parametrize("cid", [1])
 def test_layer_same_output_with_and_without_fold(cid):
-    cfg = inputs.CONFIGS[cid]
+    cfg = inputs.WORKLOADS[cid]
     d = inputs.make_inputs(cfg, DEV)
     args = (d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"], cfg.eps, cfg.K, cfg.B)
     out_fold = moe.layer(*args).clone()

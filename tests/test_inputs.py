@@ -14,7 +14,7 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 def test_deterministic_and_shapes():
-    cfg = inputs.CONFIGS[0]
+    cfg = inputs.WORKLOADS[0]
     a = inputs.make_inputs(cfg)
     b = inputs.make_inputs(cfg)
     for k in a:
@@ -26,7 +26,7 @@ def test_deterministic_and_shapes():
 
 
 def test_distributions():
-    cfg = inputs.CONFIGS[0].with_(M=256, H=1024, I=512, E=4, bias="normal", seed=5)
+    cfg = inputs.WORKLOADS[0].with_(M=256, H=1024, I=512, E=4, bias="normal", seed=5)
     a = inputs.make_inputs(cfg)
     assert abs(a["x"].float().std().item() - 1.0) < 0.02
     assert abs(a["w_router"].float().std().item() * np.sqrt(cfg.H) - 1.0) < 0.03
@@ -36,7 +36,7 @@ def test_distributions():
 
 
 def test_router_side_independent_of_expert_draws():
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.WORKLOADS[1]
     w_r, b, g, x = inputs.router_inputs(cfg)
     assert x.shape == (8, 7168) and b.shape == (256,)
     assert 0.2 < b.std().item() < 0.45   # N(0, 0.1): std ~ 0.316
@@ -51,7 +51,7 @@ def test_zipf_alpha_matches_calibration():
 
 @pytest.mark.slow
 def test_zipf_ratio_reproduced_by_oracle():
-    cfg = inputs.CONFIGS[3]
+    cfg = inputs.WORKLOADS[3]
     w_r, b, g, x = inputs.router_inputs(cfg)
     ids, _ = oracle.route(bf16_bits(x), bf16_bits(w_r), b.numpy(), cfg.K)
     counts = np.bincount(ids.ravel(), minlength=cfg.E)

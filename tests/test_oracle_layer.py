@@ -41,7 +41,7 @@ def _ulp_diff(a_bits, b_bits):
 
 
 def test_single_expert_equals_torch_swiglu_rmsnorm():
-    cfg = inputs.CONFIGS[0].with_(E=1, K=1, M=8, H=256, I=128, seed=21)
+    cfg = inputs.WORKLOADS[0].with_(E=1, K=1, M=8, H=256, I=128, seed=21)
     d = _np_inputs(cfg)
     r = oracle.layer(d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"],
                      cfg.eps, cfg.K, want_h=True)
@@ -69,7 +69,7 @@ def test_single_expert_equals_torch_swiglu_rmsnorm():
 
 
 def test_sparse_equals_dense_mixture():
-    cfg = inputs.CONFIGS[0]
+    cfg = inputs.WORKLOADS[0]
     d = _np_inputs(cfg)
     r = oracle.layer(d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"],
                      cfg.eps, cfg.K)
@@ -82,7 +82,7 @@ def test_sparse_equals_dense_mixture():
 
 
 def test_k_equals_e_is_dense_mixture():
-    cfg = inputs.CONFIGS[0].with_(E=4, K=4, M=6, seed=22, bias="normal")
+    cfg = inputs.WORKLOADS[0].with_(E=4, K=4, M=6, seed=22, bias="normal")
     d = _np_inputs(cfg)
     r = oracle.layer(d["x"], d["w_router"], d["bias"], d["w_gate"], d["w_up"], d["w_down"], d["gamma"],
                      cfg.eps, cfg.K)

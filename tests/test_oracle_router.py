@@ -62,7 +62,7 @@ def test_fma_within_lane_and_bias_last():
 
 
 def test_logit_error_bound_random():
-    cfg = inputs.CONFIGS[0].with_(M=32, H=1024, E=16)
+    cfg = inputs.WORKLOADS[0].with_(M=32, H=1024, E=16)
     w_router, bias, gamma, x = inputs.router_inputs(cfg)
     z32, z64 = oracle.router_logits(bf16_bits(x), bf16_bits(w_router), bias.numpy(), want_f64=True)
     xd, wd = bits_to_f64(bf16_bits(x)), bits_to_f64(bf16_bits(w_router))
@@ -87,7 +87,7 @@ def _valid_topk_set(z, S, K):
 
 
 def test_topk_exhaustive_tiny():
-    cfg = inputs.CONFIGS[0]
+    cfg = inputs.WORKLOADS[0]
     w_router, bias, gamma, x = inputs.router_inputs(cfg)
     z = oracle.router_logits(bf16_bits(x), bf16_bits(w_router), bias.numpy())
     ids, w = oracle.topk(z, cfg.K)
@@ -123,7 +123,7 @@ def test_weights_sum_order_and_ratio():
 
 def test_route_all_configs_shapes_small():
     # the canonical order needs H % 256 == 0; every workload satisfies it
-    for cfg in inputs.CONFIGS.values():
+    for cfg in inputs.WORKLOADS.values():
         assert cfg.H % 256 == 0 and cfg.K <= cfg.E
 
 
@@ -156,7 +156,7 @@ def test_sigmoid_without_renormalisation_is_the_score():
 def test_selection_only_bias():
     # The bias shifts which experts are picked but not their weights: the picked set is the one the
     # biased logit picks, and the weights are the renormalised sigmoid of the unbiased logit.
-    cfg = inputs.CONFIGS[0].with_(M=24, H=512, E=32, K=4)
+    cfg = inputs.WORKLOADS[0].with_(M=24, H=512, E=32, K=4)
     w_router, bias, gamma, x = inputs.router_inputs(cfg)
     b = (np.arange(cfg.E, dtype=np.float32) - cfg.E / 2) * 0.25   # large enough to change the picks
     ids, w = oracle.route_ex(bf16_bits(x), bf16_bits(w_router), b, cfg.K, bias_in_score=False)

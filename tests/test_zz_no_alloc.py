@@ -37,7 +37,7 @@ def _noalloc(x, w_router, bias, K):
 
 
 def test_route_noalloc_matches_route_on_two_calls():
-    cases = [inputs.CONFIGS[1], inputs.CONFIGS[0].with_(M=37, H=1024, E=64, K=8, bias="normal", seed=9)]
+    cases = [inputs.WORKLOADS[1], inputs.WORKLOADS[0].with_(M=37, H=1024, E=64, K=8, bias="normal", seed=9)]
     for cfg in cases:  # two calls in a row; the second reuses the array the first wrote
         w_r, b, _, x = inputs.router_inputs(cfg)
         x, w_r, b = x.cuda(), w_r.cuda(), b.cuda()
