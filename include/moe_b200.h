@@ -228,11 +228,15 @@ MOE_API moe_status_t moe_finalize_rmsnorm(const moe_bf16_t* x, const moe_bf16_t*
 
 /* ---------------------------------------------------------------- layer --
  * The whole layer on one stream: route -> align -> up -> down -> finalize
- * (flashinfer PR #6511 analysis, §6 route chain).  Intermediates live in ws
- * (moe_layer_workspace_size bytes, 256-byte aligned); the first int32 of ws
- * is the layer's device error word (cleared by each call; read it with
- * moe_get_device_error((const int32_t*)ws, ...)).  topk_ids_out / topk_w_out
- * (nullable) receive the routing.  residual_out is nullable. */
+ * (flashinfer PR #6511 analysis, §6 route chain), with the same results as
+ * calling those entry points in turn.  On decode shapes (MOE_W_BF16, at most
+ * 24 routed rows per expert on average, M*top_k <= MOE_ROUTED_UP_MAX_SLOTS)
+ * the align step runs inside the up projection (moe_grouped_up_swiglu_routed).
+ * Intermediates live in ws (moe_layer_workspace_size bytes, 256-byte aligned);
+ * the first int32 of ws is the layer's device error word (cleared by each
+ * call; read it with moe_get_device_error((const int32_t*)ws, ...)).
+ * topk_ids_out / topk_w_out (nullable) receive the routing.  residual_out is
+ * nullable.  All work is enqueued on `stream` (capturable in a CUDA graph). */
 MOE_API moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
                        const moe_weights_t* w, const moe_bf16_t* gamma, float eps, moe_shape_t s,
                        moe_bf16_t* out, moe_bf16_t* residual_out, int32_t* topk_ids_out, float* topk_w_out,
