@@ -39,6 +39,7 @@
 // and both CTAs still meet at the final cluster barrier.
 #include "common.cuh"
 #include "kernels.h"
+#include "tile_list.cuh"
 
 namespace moe {
 namespace {
@@ -133,30 +134,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
-struct TileCoord {
-  int e, w, t;
-};
-
-template <int kNmax>
-__device__ __forceinline__ TileCoord decode_tile(const int* prefix, const int* cnt, int E, int idx) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= idx) lo = mid; else hi = mid - 1;
-  }
-  const int ntiles = (cnt[lo] + kNmax - 1) / kNmax;
-  const int rel = idx - prefix[lo];
-  return TileCoord{lo, rel / ntiles, rel % ntiles};
-}
-
-template <int kN>
-__device__ __forceinline__ int pick(const int (&ids)[kN], int i) {
-  int v = ids[0];
-#pragma unroll
-  for (int j = 1; j < kN; ++j) v = (i == j) ? ids[j] : v;
-  return v;
-}
-
 template <bool kUp, int kNmax, int kStagesA, int kStagesB>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
@@ -190,24 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = tid; e < E; e += kThreads) cnt[e] = args.expert_counts[e];
   if (tid == 0) *abort_flag = 0;
   __syncthreads();
-  if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int lo = min(E, lane * per), hi = min(E, lo + per);
-    int sum = 0;
-    for (int e = lo; e < hi; ++e) sum += W * ((cnt[e] + kNmax - 1) / kNmax);
-    int incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    int run = incl - sum;
-    for (int e = lo; e < hi; ++e) {
-      prefix[e] = run;
-      run += W * ((cnt[e] + kNmax - 1) / kNmax);
-    }
-    if (lane == 31) prefix[E] = incl;
-  }
+  if (warp == 0) build_tile_prefix<kNmax>(cnt, prefix, E, W, lane);
   if (tid == 0) {
     for (int s = 0; s < kStagesA; ++s) {
       mbar_init(&a_full[s], 1);

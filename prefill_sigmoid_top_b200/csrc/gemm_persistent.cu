@@ -36,6 +36,7 @@
 // bounded.
 #include "common.cuh"
 #include "kernels.h"
+#include "tile_list.cuh"
 
 namespace moe {
 namespace {
@@ -62,33 +63,6 @@ struct PCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kSmem > 116 * 1024, "one CTA per SM: it owns all 512 tensor-memory columns");
 };
-
-struct TileCoord {
-  int e, w, t;
-};
-
-// ids[i] for a run-time i without indexing a register array.
-template <int kN>
-__device__ __forceinline__ int pick(const int (&ids)[kN], int i) {
-  int v = ids[0];
-#pragma unroll
-  for (int j = 1; j < kN; ++j) v = (i == j) ? ids[j] : v;
-  return v;
-}
-
-// Tile index -> (expert, weight tile, token tile), from prefix[e] = first tile
-// index of expert e (prefix[E] = total).  Largest e with prefix[e] <= idx.
-template <int kNmax>
-__device__ __forceinline__ TileCoord decode_tile(const int* prefix, const int* cnt, int E, int idx) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= idx) lo = mid; else hi = mid - 1;
-  }
-  const int ntiles = (cnt[lo] + kNmax - 1) / kNmax;
-  const int rel = idx - prefix[lo];
-  return TileCoord{lo, rel / ntiles, rel % ntiles};
-}
 
 // kGatherB (up only): the token-row producer gathers the rows of x itself
 // with tile::gather4 (x stays in L2); otherwise tm_b maps a plan-ordered
@@ -123,24 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = tid; e < E; e += kThreads) cnt[e] = args.expert_counts[e];
   if (tid == 0) *abort_flag = 0;
   __syncthreads();
-  if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int lo = min(E, lane * per), hi = min(E, lo + per);
-    int sum = 0;
-    for (int e = lo; e < hi; ++e) sum += W * ((cnt[e] + kNmax - 1) / kNmax);
-    int incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    int run = incl - sum;
-    for (int e = lo; e < hi; ++e) {
-      prefix[e] = run;
-      run += W * ((cnt[e] + kNmax - 1) / kNmax);
-    }
-    if (lane == 31) prefix[E] = incl;
-  }
+  if (warp == 0) build_tile_prefix<kNmax>(cnt, prefix, E, W, lane);
   if (tid == 0) {
     for (int s = 0; s < kStagesA; ++s) {
       mbar_init(&a_full[s], 1);

@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tile_list.cuh"
 
 namespace moe {
 namespace {
@@ -319,21 +320,6 @@ static_assert(kSmem <= 227 * 1024, "shared memory");
 static_assert(kSmem > 116 * 1024, "one CTA per SM");
 static_assert(2 * kNmax + kSfSlots * kSfCols <= 512, "tensor memory");
 
-struct TileCoord {
-  int e, w, t;
-};
-
-__device__ __forceinline__ TileCoord decode_tile(const int* prefix, const int* cnt, int E, int idx) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= idx) lo = mid; else hi = mid - 1;
-  }
-  const int ntiles = (cnt[lo] + kNmax - 1) / kNmax;
-  const int rel = idx - prefix[lo];
-  return TileCoord{lo, rel / ntiles, rel % ntiles};
-}
-
 template <bool kUp>
 __global__ void __launch_bounds__(kThreads, 1)
     persistent_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
@@ -364,24 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = tid; e < E; e += kThreads) cnt[e] = g.expert_counts[e];
   if (tid == 0) *abort_flag = 0;
   __syncthreads();
-  if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int lo = min(E, lane * per), hi = min(E, lo + per);
-    int sum = 0;
-    for (int e = lo; e < hi; ++e) sum += W * ((cnt[e] + kNmax - 1) / kNmax);
-    int incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    int run = incl - sum;
-    for (int e = lo; e < hi; ++e) {
-      prefix[e] = run;
-      run += W * ((cnt[e] + kNmax - 1) / kNmax);
-    }
-    if (lane == 31) prefix[E] = incl;
-  }
+  if (warp == 0) build_tile_prefix<kNmax>(cnt, prefix, E, W, lane);
   if (tid == 0) {
     for (int s = 0; s < kStagesA; ++s) {
       mbar_init(&a_full[s], 1);
@@ -421,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ka = 0;
     bool alive = true;
     for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
-      const TileCoord c = decode_tile(prefix, cnt, E, tile);
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
       const uint64_t pol = cnt[c.e] <= kNmax ? l2_policy_evict_first() : l2_policy_evict_normal();
       const int row_a0 = kUp ? c.e * g.rows_per_expert + c.w * kBM : c.e * g.rows_per_expert + c.w * 2 * kBM;
       const int row_a1 = kUp ? row_a0 : row_a0 + kBM;
@@ -460,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kb = 0;
     bool alive = true;
     for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x) {
-      const TileCoord c = decode_tile(prefix, cnt, E, tile);
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
       const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
       const int ti = prefix[c.e] / W + c.t;  // global token-tile index
       const int nbox = (nrows + kBRows - 1) / kBRows;
@@ -495,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ka = 0, kb = 0, j = 0, step = 0;
       bool alive = true;
       for (int tile = blockIdx.x; tile < total && alive; tile += gridDim.x, ++j) {
-        const TileCoord c = decode_tile(prefix, cnt, E, tile);
+        const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
         const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
         const int N = (nrows + 15) & ~15;
         const uint32_t idesc = umma_idesc_nvfp4(kBM, N);
@@ -582,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float hmax = 0.0f;  // up: max |h| of the values this thread stores
     int j = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
-      const TileCoord c = decode_tile(prefix, cnt, E, tile);
+      const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
       const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
       const int N = (nrows + 15) & ~15;
       const int row0 = g.expert_offsets[c.e] + c.t * kNmax;
