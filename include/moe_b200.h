@@ -18,7 +18,8 @@
  *                intermediate in HBM ("[flashinfer] Kimi K3를 위한 초고속 통신
  *                최적화", flashinfer PR #5701 analysis, intro and §2 HT preset:
  *                H=7168 = 896 bf16x8 packs; §3: RMS_EPS=1e-5, WEIGHT_BIAS=0).
- *   moe_layer    runs 1-5 on one stream (PR #6511 analysis, §6 route chain).
+ *   moe_layer    runs 1-5 on one stream (PR #6511 analysis, §6 route chain);
+ *                on decode shapes as a single launch.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -34,7 +35,9 @@
  *    never trap: the kernel ORs a bit into the int32 word at `err_flag`
  *    (nullable: then they are silently ignored) and the affected outputs are
  *    unspecified.  Read it with moe_get_device_error().  Bit (1 << status)
- *    is set for status MOE_ERR_INVALID_INPUT or MOE_ERR_TIMEOUT.
+ *    is set for status MOE_ERR_INVALID_INPUT or MOE_ERR_TIMEOUT, or
+ *    MOE_ERR_UNSUPPORTED for a launch the kernel found it cannot run (the
+ *    single-launch layer given shared memory without 1024-byte alignment).
  *  - Waits inside kernels are bounded (0.5 s each); on expiry the kernel
  *    sets the MOE_ERR_TIMEOUT bit and returns.
  *  - Accepted shapes: M >= 1; H % 256 == 0 and H <= 8192; I % 128 == 0
@@ -230,8 +233,15 @@ MOE_API moe_status_t moe_finalize_rmsnorm(const moe_bf16_t* x, const moe_bf16_t*
  * The whole layer on one stream: route -> align -> up -> down -> finalize
  * (flashinfer PR #6511 analysis, §6 route chain), with the same results as
  * calling those entry points in turn.  On decode shapes (MOE_W_BF16, at most
- * 24 routed rows per expert on average, M*top_k <= MOE_ROUTED_UP_MAX_SLOTS)
- * the align step runs inside the up projection (moe_grouped_up_swiglu_routed).
+ * 24 routed rows per expert on average, M*top_k <= MOE_ROUTED_UP_MAX_SLOTS,
+ * E <= 256) the layer is ONE cooperative launch (one CTA pair per SM: the
+ * router, a grid barrier, the plan, the up and down tiles handed out by a
+ * device-side counter with the down tiles of an expert waiting for its up
+ * tiles, then the finalize; the megakernel of "AWS Trainium2에서 GLM-5.3-Flash를
+ * 위한 NKI 레이어 메가커널"), bit-identical to the separate entry points;
+ * MOE_FUSED_LAYER=0 in the environment selects the 5-launch form instead, in
+ * which the align step runs inside the up projection
+ * (moe_grouped_up_swiglu_routed).
  * Intermediates live in ws (moe_layer_workspace_size bytes, 256-byte aligned);
  * the first int32 of ws is the layer's device error word (cleared by each
  * call; read it with moe_get_device_error((const int32_t*)ws, ...)).
@@ -251,7 +261,9 @@ MOE_API int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype);
 /* Byte offsets of the layer's intermediates inside ws (for inspection). */
 typedef struct {
   size_t err_flag, logits, topk_ids, topk_w, sorted_ids, block_expert, expert_counts, expert_offsets,
-      num_tokens_post_padded, h, y, act_scratch, total;
+      num_tokens_post_padded, h, y, act_scratch,
+      sync, /* 3 + E uint32 counters of the single-launch layer, cleared with the error word */
+      total;
 } moe_layer_ws_layout_t;
 MOE_API moe_status_t moe_layer_workspace_layout(moe_shape_t s, moe_wdtype_t dtype, moe_layer_ws_layout_t* layout);
 
@@ -311,7 +323,8 @@ MOE_API moe_status_t moe_route_noalloc(const moe_bf16_t* x, const moe_bf16_t* w_
 /* ---------------------------------------------------------------- errors -
  * Synchronises `stream`, reads the device error word and returns, in
  * *host_code, MOE_OK or the most severe device-detected status
- * (MOE_ERR_TIMEOUT before MOE_ERR_INVALID_INPUT).  Clears nothing. */
+ * (MOE_ERR_TIMEOUT before MOE_ERR_INVALID_INPUT before MOE_ERR_UNSUPPORTED).
+ * Clears nothing. */
 MOE_API moe_status_t moe_get_device_error(const int32_t* err_flag, moe_stream_t stream, int32_t* host_code);
 
 /* Failure-path self-test: launches one warp whose bounded wait (the same wait

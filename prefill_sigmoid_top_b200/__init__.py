@@ -64,7 +64,7 @@ class _RouteOpts(ctypes.Structure):
 SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
 
 _LAYOUT_FIELDS = ["err_flag", "logits", "topk_ids", "topk_w", "sorted_ids", "block_expert", "expert_counts",
-                  "expert_offsets", "num_tokens_post_padded", "h", "y", "act_scratch", "total"]
+                  "expert_offsets", "num_tokens_post_padded", "h", "y", "act_scratch", "sync", "total"]
 
 
 class _Layout(ctypes.Structure):

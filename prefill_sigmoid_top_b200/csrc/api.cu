@@ -284,6 +284,55 @@ bool want_self_route(const moe_shape_t& s, moe_wdtype_t dt) {
          static_cast<long long>(s.M) * s.top_k <= moe::kRouteMaxSlots;
 }
 
+// Whether moe_layer runs as one launch (layer_fused.cu): the decode shapes of
+// the self-routing path with at most 256 experts.  MOE_FUSED_LAYER=0 turns it
+// off (the tests cover both).
+bool want_fused_layer(const moe_shape_t& s, moe_wdtype_t dt) {
+  if (const char* env = std::getenv("MOE_FUSED_LAYER"))
+    if (std::strcmp(env, "0") == 0) return false;
+  return want_self_route(s, dt) && s.E <= 256;
+}
+
+moe_status_t run_layer_fused(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                             const moe_weights_t* w, const moe_bf16_t* gamma, float eps, const moe_shape_t& s,
+                             moe_bf16_t* out, moe_bf16_t* residual_out, int32_t* ids, float* tw, uint8_t* base,
+                             const moe_layer_ws_layout_t& L, cudaStream_t stream) {
+  CUtensorMap mg, mu, md, mx, mh;
+  const uint64_t rows = static_cast<uint64_t>(s.E) * s.I;
+  auto* h = reinterpret_cast<moe_bf16_t*>(base + L.h);
+  if (!make_map_bf16(&mg, w->gate, rows, s.H, 128) || !make_map_bf16(&mu, w->up, rows, s.H, 128) ||
+      !make_map_bf16(&md, w->down, static_cast<uint64_t>(s.E) * s.H, s.I, 128) ||
+      !make_map_bf16(&mx, x, s.M, s.H, 1) || !make_map_bf16(&mh, h, cap_rows(s), s.I, 16))
+    return MOE_ERR_CUDA;
+  moe::FusedLayerArgs a{};
+  a.x = x;
+  a.w_router = w_router;
+  a.bias = bias;
+  a.gamma = gamma;
+  a.eps = eps;
+  a.M = s.M;
+  a.H = s.H;
+  a.I = s.I;
+  a.E = s.E;
+  a.top_k = s.top_k;
+  a.block_size = s.block_size;
+  a.logits = reinterpret_cast<float*>(base + L.logits);
+  a.topk_ids = ids;
+  a.topk_w = tw;
+  a.sorted_ids = reinterpret_cast<int32_t*>(base + L.sorted_ids);
+  a.block_expert = reinterpret_cast<int32_t*>(base + L.block_expert);
+  a.counts = reinterpret_cast<int32_t*>(base + L.expert_counts);
+  a.offsets = reinterpret_cast<int32_t*>(base + L.expert_offsets);
+  a.ntpp = reinterpret_cast<int32_t*>(base + L.num_tokens_post_padded);
+  a.h = h;
+  a.y = reinterpret_cast<moe_bf16_t*>(base + L.y);
+  a.out = out;
+  a.residual_out = residual_out;
+  a.err = reinterpret_cast<int32_t*>(base + L.err_flag);
+  a.sync = reinterpret_cast<unsigned*>(base + L.sync);
+  return cuda_status(moe::launch_layer_fused(mg, mu, md, mx, mh, a, num_sms(), stream));
+}
+
 moe_status_t run_up_routed(const moe_bf16_t* x, const moe_weights_t* w, const int32_t* topk_ids,
                            const moe_shape_t& s, int32_t* sorted_ids, int32_t* block_expert, int32_t* counts,
                            int32_t* offsets, int32_t* ntpp, moe_bf16_t* h, int32_t* err, cudaStream_t stream) {
@@ -428,7 +477,8 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   const size_t cap = cap_rows(s);
   size_t off = 0;
   L.err_flag = off;
-  off += kAlign;
+  L.sync = off + 16;  // zeroed with the error word before every layer call
+  off = align_up(L.sync + (3 + static_cast<size_t>(s.E)) * sizeof(uint32_t));
   L.logits = off;
   off = align_up(off + static_cast<size_t>(s.M) * s.E * sizeof(float));
   L.topk_ids = off;
@@ -661,7 +711,10 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   auto* h = reinterpret_cast<moe_bf16_t*>(base + L.h);
   auto* y = reinterpret_cast<moe_bf16_t*>(base + L.y);
 
-  if ((st = cuda_status(cudaMemsetAsync(err, 0, sizeof(int32_t), cs))) != MOE_OK) return st;
+  // the error word and the single-launch layer's counters, in one region
+  if ((st = cuda_status(cudaMemsetAsync(err, 0, L.logits - L.err_flag, cs))) != MOE_OK) return st;
+  if (want_fused_layer(s, w->dtype))
+    return run_layer_fused(x, w_router, bias, w, gamma, eps, s, out, residual_out, ids, tw, base, L, cs);
   float* logits = reinterpret_cast<float*>(base + L.logits);
   if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
     return st;
@@ -694,7 +747,8 @@ int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK || (dtype != MOE_W_BF16 && dtype != MOE_W_NVFP4)) return -1;
   if (dtype == MOE_W_NVFP4)  // router x2, align, amax x, quantize x, gather tiles, up (+ amax h), quantize h, down, finalize
     return 10;
-  if (want_self_route(s, dtype)) return 5;  // router x2, up with the plan, down, finalize
+  if (want_fused_layer(s, dtype)) return 1;  // the whole layer in one launch
+  if (want_self_route(s, dtype)) return 5;   // router x2, up with the plan, down, finalize
   return 6 + (want_pregather(s) ? 1 : 0);   // router x2, align, [gather x], up, down, finalize
 }
 
@@ -752,6 +806,8 @@ moe_status_t moe_get_device_error(const int32_t* err_flag, moe_stream_t stream, 
     *host_code = MOE_ERR_TIMEOUT;
   else if (v & moe::kErrInvalidInput)
     *host_code = MOE_ERR_INVALID_INPUT;
+  else if (v & moe::kErrUnsupported)
+    *host_code = MOE_ERR_UNSUPPORTED;
   else
     *host_code = MOE_OK;
   return MOE_OK;

@@ -100,6 +100,44 @@ cudaError_t launch_persistent_up(const CUtensorMap& w_gate, const CUtensorMap& w
 cudaError_t launch_persistent_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
                                    int nmax, bool deep_b, int num_sms, cudaStream_t stream);
 
+// Device error bit of a kernel that cannot run as launched (layer_fused.cu:
+// a dynamic shared-memory base that is not 1024-byte aligned): MOE_ERR_UNSUPPORTED.
+constexpr int32_t kErrUnsupported = 1 << 2;
+
+// layer_fused.cu: the decode-shaped layer (route, plan, up, down, finalize)
+// in one cooperative launch.  `sync` points at 3 + E words that are zero when
+// the launch starts: grid barrier, work counter, finalize count, and one
+// up-tile count per expert.
+struct FusedLayerArgs {
+  const uint16_t* x;         // [M, H]
+  const uint16_t* w_router;  // [E, H]
+  const float* bias;         // [E] or null
+  const uint16_t* gamma;     // [H]
+  float eps;
+  int M, H, I, E, top_k, block_size;
+  float* logits;             // [M, E] scratch
+  int32_t* topk_ids;         // [M, top_k]
+  float* topk_w;             // [M, top_k]
+  int32_t* sorted_ids;       // the plan, as moe_align_block_size writes it
+  int32_t* block_expert;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* ntpp;
+  uint16_t* h;               // [cap, I]
+  uint16_t* y;               // [M*top_k, H]
+  uint16_t* out;             // [M, H]
+  uint16_t* residual_out;    // [M, H] or null
+  int32_t* err;
+  unsigned* sync;
+};
+// Tensor maps: W_gate / W_up as [E*I, H] and W_down as [E*H, I] in 128-row
+// boxes, x as [M, H] in one-row boxes (tile::gather4), h as [cap, I] in
+// 16-row boxes.
+cudaError_t launch_layer_fused(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& w_down,
+                               const CUtensorMap& x_rows, const CUtensorMap& h_rows, const FusedLayerArgs& args,
+                               int num_sms, cudaStream_t stream);
+int layer_fused_smem_bytes(int E, int nslots);
+
 // nvfp4.cu ------------------------------------------------------------------
 struct Nvfp4GemmArgs {
   GroupedGemmArgs g;      // kdim in elements; out / plan / shape as for bf16

@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "router_dot.cuh"
 
 namespace moe {
 namespace {
@@ -63,30 +64,6 @@ struct StagedCfg {
   static_assert((kRows * 32) % kThreads == 0, "copy split");
   static_assert(kTt * kTe <= 64, "pairs per warp");
 };
-
-// fp32 fma with bf16 multiplicands: c + a*b rounded once, a and b taken
-// exactly (a product of two bf16 values is exact in fp32), so the result is
-// the same as fmaf(float(a), float(b), c) without the two conversions.
-// kHi selects the high or the low bf16 half of each 32-bit word.
-template <bool kHi>
-__device__ __forceinline__ float fma_bf16(uint32_t aw, uint32_t bw, float c) {
-  float d = c;
-  if (kHi)
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
-        : "+f"(d)
-        : "r"(aw), "r"(bw));
-  else
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t}"
-        : "+f"(d)
-        : "r"(aw), "r"(bw));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t word(const uint4& v, int w) {
-  return w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
-}
 
 template <int kTt, int kTe, int kWt, int kWe, int kStages>
 __global__ void __launch_bounds__(kWt * kWe * 32) router_logits_staged_kernel(const uint16_t* __restrict__ x,

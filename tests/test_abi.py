@@ -146,8 +146,13 @@ def test_routed_up_rejects_bad_arguments():
     assert L.moe_grouped_up_swiglu_routed(*a) == 1
 
 
-def test_layer_kernel_count():
-    assert moe.layer_kernel_count(C1) == 5            # decode: align folded into the up kernel
+def test_layer_kernel_count(monkeypatch):
+    assert moe.layer_kernel_count(C1) == 1            # decode: the whole layer in one launch
+    monkeypatch.setenv("MOE_FUSED_LAYER", "0")
+    assert moe.layer_kernel_count(C1) == 5            # decode, separate launches: align folded into up
+    monkeypatch.delenv("MOE_FUSED_LAYER")
+    many_experts = moe.Shape(M=2, H=7168, I=2048, E=512, top_k=8, block_size=16)
+    assert moe.layer_kernel_count(many_experts) == 5  # the single launch takes E <= 256
     batch = moe.Shape(M=512, H=7168, I=2048, E=256, top_k=16, block_size=64)
     assert moe.layer_kernel_count(batch) == 7         # align and a gather pass of x
     assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 10
