@@ -262,7 +262,7 @@ MOE_API int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype);
 typedef struct {
   size_t err_flag, logits, topk_ids, topk_w, sorted_ids, block_expert, expert_counts, expert_offsets,
       num_tokens_post_padded, h, y, act_scratch,
-      sync, /* 3 + E uint32 counters of the single-launch layer, cleared with the error word */
+      sync, /* uint32 counters of the single-launch layer (3 + E, + 9 M for M <= 64), cleared with the error word */
       total;
 } moe_layer_ws_layout_t;
 MOE_API moe_status_t moe_layer_workspace_layout(moe_shape_t s, moe_wdtype_t dtype, moe_layer_ws_layout_t* layout);

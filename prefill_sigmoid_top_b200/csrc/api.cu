@@ -471,6 +471,13 @@ moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const m
   return cuda_status(moe::launch_nvfp4_down(md, mh, a, num_sms(), stream));
 }
 
+// Counters of the single-launch layer: grid barrier, work counter, finalize
+// count, one up-tile count per expert, and (up to 64 tokens) one slice count
+// and 8 partial sums of squares per token.
+size_t fused_sync_words(const moe_shape_t& s) {
+  return 3 + static_cast<size_t>(s.E) + (s.M <= 64 ? 9 * static_cast<size_t>(s.M) : 0);
+}
+
 moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   moe_layer_ws_layout_t L{};
   const size_t mk = static_cast<size_t>(s.M) * s.top_k;
@@ -478,7 +485,7 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   size_t off = 0;
   L.err_flag = off;
   L.sync = off + 16;  // zeroed with the error word before every layer call
-  off = align_up(L.sync + (3 + static_cast<size_t>(s.E)) * sizeof(uint32_t));
+  off = align_up(L.sync + fused_sync_words(s) * sizeof(uint32_t));
   L.logits = off;
   off = align_up(off + static_cast<size_t>(s.M) * s.E * sizeof(float));
   L.topk_ids = off;

@@ -105,9 +105,10 @@ cudaError_t launch_persistent_down(const CUtensorMap& w_down, const CUtensorMap&
 constexpr int32_t kErrUnsupported = 1 << 2;
 
 // layer_fused.cu: the decode-shaped layer (route, plan, up, down, finalize)
-// in one cooperative launch.  `sync` points at 3 + E words that are zero when
-// the launch starts: grid barrier, work counter, finalize count, and one
-// up-tile count per expert.
+// in one cooperative launch.  `sync` points at 3 + E (+ 9 M when M <= 64)
+// words that are zero when the launch starts: grid barrier, work counter,
+// finalize count, one up-tile count per expert, then per token a count of
+// finalize slices and their 8 partial sums of squares.
 struct FusedLayerArgs {
   const uint16_t* x;         // [M, H]
   const uint16_t* w_router;  // [E, H]

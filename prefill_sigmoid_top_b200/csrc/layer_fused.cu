@@ -9,9 +9,10 @@
 // the router, same MMA shapes and K order in the projections, the finalize's
 // reduction order), on one cooperative grid of one CTA per SM:
 //
-//  1. router logits: every warp of the grid takes (4 tokens x 2 experts)
-//     items; lane l keeps partial l of each pair in the canonical order.
-//     z goes to the workspace; one bounded grid barrier.
+//  1. router logits: a CTA takes 8 tokens x 6 experts at a time, their rows
+//     staged whole in shared memory by bulk copies; lane l keeps partial l of
+//     each pair in the canonical order.  z goes to the workspace; one bounded
+//     grid barrier.
 //  2. top-k and plan, redundantly in every CTA (at most 1024 routed slots):
 //     warp-argmax top-k of every token, per-expert counts, the padded and the
 //     compact prefix, and the slot ids of every expert in ascending slot
@@ -26,8 +27,10 @@
 //     and a claimed tile never waits on a later one, so every wait ends.
 //     The down tiles of the first experts start while the last up tiles are
 //     still streaming, so no SM idles between the two projections.
-//  4. finalize + residual + RMSNorm of one token by the 4 epilogue warps, in the
-//     reduction order of the finalize kernel the separate launches would use.
+//  4. finalize + residual + RMSNorm by the 4 epilogue warps, in the reduction
+//     order of the finalize kernel the separate launches would use: up to 64
+//     tokens, 8 slices per token on 8 CTAs whose partial sums of squares meet
+//     in the workspace (added in slice order); more, one token per item.
 //
 // Warp roles in the 192-thread CTA (after phases 1-2, which all warps share):
 //   warp 0      producer: claims work, queues it for the other roles, and
@@ -67,7 +70,7 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kEpiWarp0 = 2;
 constexpr int kEpiThreads = 128;
 constexpr int kSplit = 8;                    // finalize: 8 accumulator sets of one 8-element pack
-constexpr int kRtTok = 4, kRtExp = 2;        // router item: tokens x experts per warp
+constexpr int kRtTok = 8;                    // router item: tokens (x experts, one per warp)
 constexpr int kTopkPerLane = 8;              // E <= 256
 
 enum : int { kKindUp = 0, kKindDown = 1, kKindFin = 2, kKindEnd = 3 };
@@ -76,7 +79,7 @@ enum : int { kKindUp = 0, kKindDown = 1, kKindFin = 2, kKindEnd = 3 };
 // The ring takes almost all of it, so the plan is packed: int16 wherever the
 // value fits (slot ids, compact offsets and token-tile prefixes stay below 2^15).
 constexpr int kRingOff = 0;
-constexpr int kNumBars = 2 * kSlots + 2 + 2 + 2 * kQueue + 2;
+constexpr int kNumBars = 2 * kSlots + 2 + 2 + 2 * kQueue + 3;
 constexpr int kBarOff = kSlots * kSlotBytes;
 constexpr int kWordOff = kBarOff + ((kNumBars * 8 + 15) / 16) * 16;  // tmem base, abort flag
 constexpr int kQueueOff = kWordOff + 16;                             // int4 [kQueue], then the epilogue's item
@@ -101,6 +104,9 @@ __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // Through L2 only: the data was written by other SMs during this launch.
@@ -167,9 +173,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tqe = tqf + kQueue;     // [kQueue]
   uint64_t* drain = tqe + kQueue;
   uint64_t* fin_bar = drain + 1;    // a finalize item of this CTA is done
+  uint64_t* rt_bar = fin_bar + 1;   // the router rows of an item have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kWordOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kWordOff + 4);
   volatile int* epi_go = reinterpret_cast<volatile int*>(smem + kWordOff + 8);  // epilogue group: outcome of a wait
+  volatile float* fin_total = reinterpret_cast<volatile float*>(smem + kWordOff + 12);  // a token's sum of squares
   volatile int* epi_item = reinterpret_cast<volatile int*>(smem + kQueueOff + 16 * kQueue);  // int4
   int4* queue = reinterpret_cast<int4*>(smem + kQueueOff);
   float* part = reinterpret_cast<float*>(smem + kPartOff);
@@ -188,67 +196,79 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned* next_work = args.sync + 1;
   unsigned* down_done = args.sync + 2;
   unsigned* up_done = args.sync + 3;  // [E]
+  unsigned* fin_cnt = up_done + E;     // [M] slices of a token whose partial is written (M <= 64)
+  float* fin_part = reinterpret_cast<float*>(fin_cnt + M);  // [M][8] per-slice sums of squares
   if ((smem_addr(smem_raw) & 1023u) != 0) {  // the 128-byte swizzle needs 1024-byte aligned tiles
     if (tid == 0) set_error(args.err, kErrUnsupported);
     return;
   }
 
   // ------------------------------------------------ 1. router logits
+  // A CTA item = 8 tokens x ne experts.  Their rows are copied whole into the
+  // ring with bulk copies on one mbarrier; warp w < ne then takes expert
+  // e0 + w for the 8 tokens from shared memory, lane l keeping partial l
+  // (chunks 32j + l, one fma per element in increasing h).
+  if (tid == 0) {
+    *abort_flag = 0;
+    mbar_init(rt_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
   {
-    const int tgroups = (M + kRtTok - 1) / kRtTok, egroups = (E + kRtExp - 1) / kRtExp;
+    const int row_bytes = H * 2;
+    const int ne = min(kWarps, kSlots * kSlotBytes / row_bytes - kRtTok);  // >= 5 for H <= 8192
+    const int tgroups = (M + kRtTok - 1) / kRtTok, egroups = (E + ne - 1) / ne;
     const int items = tgroups * egroups;
     const int nj = H / 256;
-    const int row_vecs = H / 8;
-    const uint4* xv4 = reinterpret_cast<const uint4*>(args.x);
-    const uint4* wv4 = reinterpret_cast<const uint4*>(args.w_router);
-    for (int it = blockIdx.x * kWarps + warp; it < items; it += gridDim.x * kWarps) {
-      const int t0 = (it / egroups) * kRtTok, e0 = (it % egroups) * kRtExp;
-      const uint4* xr[kRtTok];
-      const uint4* wr[kRtExp];
-#pragma unroll
-      for (int t = 0; t < kRtTok; ++t) xr[t] = xv4 + static_cast<size_t>(t0 + t < M ? t0 + t : 0) * row_vecs + lane;
-#pragma unroll
-      for (int q = 0; q < kRtExp; ++q) wr[q] = wv4 + static_cast<size_t>(e0 + q < E ? e0 + q : 0) * row_vecs + lane;
-      float acc[kRtTok][kRtExp];
-#pragma unroll
-      for (int t = 0; t < kRtTok; ++t)
-#pragma unroll
-        for (int q = 0; q < kRtExp; ++q) acc[t][q] = 0.0f;
-#pragma unroll 2
-      for (int j = 0; j < nj; ++j) {
-        uint4 xa[kRtTok], wa[kRtExp];
-#pragma unroll
-        for (int t = 0; t < kRtTok; ++t) xa[t] = __ldg(xr[t] + 32 * j);
-#pragma unroll
-        for (int q = 0; q < kRtExp; ++q) wa[q] = __ldg(wr[q] + 32 * j);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)  // increasing h inside the 8-element chunk
-#pragma unroll
-          for (int t = 0; t < kRtTok; ++t)
-#pragma unroll
-            for (int q = 0; q < kRtExp; ++q)
-              acc[t][q] = (i & 1) ? fma_bf16<true>(word(xa[t], i >> 1), word(wa[q], i >> 1), acc[t][q])
-                                  : fma_bf16<false>(word(xa[t], i >> 1), word(wa[q], i >> 1), acc[t][q]);
+    int round = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x, ++round) {
+      const int t0 = (it / egroups) * kRtTok, e0 = (it % egroups) * ne;
+      const int nt = min(kRtTok, M - t0), nex = min(ne, E - e0);
+      if (tid == 0) {
+        mbar_arrive_expect_tx(rt_bar, static_cast<uint32_t>((nt + nex) * row_bytes));
+        for (int r = 0; r < nt; ++r)
+          bulk_load(ring + r * row_bytes, args.x + static_cast<size_t>(t0 + r) * H, row_bytes, rt_bar);
+        for (int r = 0; r < nex; ++r)
+          bulk_load(ring + (kRtTok + r) * row_bytes, args.w_router + static_cast<size_t>(e0 + r) * H, row_bytes,
+                    rt_bar);
       }
+      if (!mbar_wait_bounded(rt_bar, round & 1, nullptr)) {
+        *abort_flag = 1;
+        set_error(args.err, kErrTimeout);
+      } else if (warp < nex) {
+        const uint4* wrow = reinterpret_cast<const uint4*>(ring + (kRtTok + warp) * row_bytes) + lane;
+        const uint4* xrow = reinterpret_cast<const uint4*>(ring) + lane;
+        const int rv = row_bytes / 16;
+        float acc[kRtTok];
 #pragma unroll
-      for (int t = 0; t < kRtTok; ++t)
+        for (int t = 0; t < kRtTok; ++t) acc[t] = 0.0f;
+#pragma unroll 2
+        for (int j = 0; j < nj; ++j) {
+          const uint4 wa = wrow[32 * j];
 #pragma unroll
-        for (int q = 0; q < kRtExp; ++q) {
-          float v = acc[t][q];
+          for (int t = 0; t < kRtTok; ++t) {
+            const uint4 xa = xrow[t * rv + 32 * j];
 #pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
-          const int tok = t0 + t, e = e0 + q;
-          if (lane == 0 && tok < M && e < E) {
-            const float b = args.bias != nullptr ? args.bias[e] : 0.0f;
-            args.logits[static_cast<size_t>(tok) * E + e] = __fadd_rn(v, b);
+            for (int i = 0; i < 8; ++i)  // increasing h inside the 8-element chunk
+              acc[t] = (i & 1) ? fma_bf16<true>(word(xa, i >> 1), word(wa, i >> 1), acc[t])
+                               : fma_bf16<false>(word(xa, i >> 1), word(wa, i >> 1), acc[t]);
           }
         }
+        const int e = e0 + warp;
+        const float b = args.bias != nullptr ? args.bias[e] : 0.0f;
+#pragma unroll
+        for (int t = 0; t < kRtTok; ++t) {
+          float v = acc[t];
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+          if (lane == 0 && t < nt) args.logits[static_cast<size_t>(t0 + t) * E + e] = __fadd_rn(v, b);
+        }
+      }
+      __syncthreads();  // the rows may be replaced by the next item's copies
     }
   }
   // grid barrier: every logit is written (the counter was zeroed before the launch)
-  __syncthreads();
   if (tid == 0) {
-    *abort_flag = 0;
     __threadfence();
     atomicAdd(bar_word, 1u);
     if (!wait_count(bar_word, gridDim.x, nullptr)) {
@@ -263,52 +283,69 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* ids_s = reinterpret_cast<int*>(ring);  // [nslots] scratch in the ring
   int* run = ids_s + nslots;                  // [E] scratch
   int* cnt_s = run + E;                       // [E] scratch
-  for (int t = warp; t < M; t += kWarps) {
-    float v[kTopkPerLane];
-    bool live[kTopkPerLane];
+  // Two tokens per warp at a time (t and t + kWarps), their selections
+  // interleaved so that the two dependent chains overlap; each token takes
+  // exactly the steps of the router's top-k kernel.
+  for (int t = warp; t < M; t += 2 * kWarps) {
+    const int tt[2] = {t, t + kWarps};
+    float v[2][kTopkPerLane];
+    bool live[2][kTopkPerLane];
 #pragma unroll
-    for (int i = 0; i < kTopkPerLane; ++i) {
-      const int e = lane + 32 * i;
-      live[i] = e < E;
-      v[i] = live[i] ? ld_cg_f32(args.logits + static_cast<size_t>(t) * E + e) : -INFINITY;
-    }
-    float sel_v = 0.0f;
-    int sel_id = 0;
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < kTopkPerLane; ++i) {
+        const int e = lane + 32 * i;
+        live[u][i] = e < E && tt[u] < M;
+        v[u][i] = live[u][i] ? ld_cg_f32(args.logits + static_cast<size_t>(tt[u]) * E + e) : -INFINITY;
+      }
+    float sel_v[2] = {0.0f, 0.0f};
+    int sel_id[2] = {0, 0};
     for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+      float bv[2] = {-INFINITY, -INFINITY};
+      int bi[2] = {0x7fffffff, 0x7fffffff};
 #pragma unroll
-      for (int i = 0; i < kTopkPerLane; ++i)
-        if (live[i] && better(v[i], lane + 32 * i, bv, bi)) {
-          bv = v[i];
-          bi = lane + 32 * i;
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int i = 0; i < kTopkPerLane; ++i)
+          if (live[u][i] && better(v[u][i], lane + 32 * i, bv[u], bi[u])) {
+            bv[u] = v[u][i];
+            bi[u] = lane + 32 * i;
+          }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv[u], off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi[u], off);
+          if (better(ov, oi, bv[u], bi[u])) {
+            bv[u] = ov;
+            bi[u] = oi;
+          }
         }
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
+      for (int u = 0; u < 2; ++u) {
 #pragma unroll
-      for (int i = 0; i < kTopkPerLane; ++i)
-        if (lane + 32 * i == bi) live[i] = false;
-      if (lane == k) {
-        sel_v = bv;
-        sel_id = bi;
+        for (int i = 0; i < kTopkPerLane; ++i)
+          if (lane + 32 * i == bi[u]) live[u][i] = false;
+        if (lane == k) {
+          sel_v[u] = bv[u];
+          sel_id[u] = bi[u];
+        }
       }
     }
-    const float s = (lane < K) ? 1.0f / (1.0f + expf(-sel_v)) : 0.0f;
-    float total = s;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
-    if (lane < K) {
-      ids_s[t * K + lane] = sel_id;
-      if (blockIdx.x == 0) {
-        args.topk_ids[static_cast<size_t>(t) * K + lane] = sel_id;
-        args.topk_w[static_cast<size_t>(t) * K + lane] = s / total;
+    for (int u = 0; u < 2; ++u) {
+      if (tt[u] >= M) break;
+      const float sv = (lane < K) ? 1.0f / (1.0f + expf(-sel_v[u])) : 0.0f;
+      float total = sv;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+      if (lane < K) {
+        ids_s[tt[u] * K + lane] = sel_id[u];
+        if (blockIdx.x == 0) {
+          args.topk_ids[static_cast<size_t>(tt[u]) * K + lane] = sel_id[u];
+          args.topk_w[static_cast<size_t>(tt[u]) * K + lane] = sv / total;
+        }
       }
     }
   }
@@ -392,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  fence_proxy_async_shared();  // the scratch writes above come before the ring's TMA writes
   tc_fence_before_sync();
   __syncthreads();  // the plan is complete; the ring scratch is free again
   tc_fence_after_sync();
@@ -424,7 +462,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Wu = I / kBM, Wd = H / (2 * kBM);
   const int ntiles = tp[E];
   const int n_up = Wu * ntiles, n_down = Wd * ntiles;
-  const int n_work = n_up + n_down + M;
+  // finalize items: 8 slices per token up to 64 tokens (as the few-token
+  // finalize kernel's 8-CTA clusters), else one item per token
+  const bool split_fin = M <= 64;
+  const int n_fin = split_fin ? M * kSplit : M;
+  const int n_work = n_up + n_down + n_fin;
 
   if (warp == 0) {
     // ------------------------------------------------ producer
@@ -458,7 +500,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int4 w;
       if (q < n_up) w = decode_work(tp, E, Wu, q, kKindUp);
       else if (q < n_up + n_down) w = decode_work(tp, E, Wd, q - n_up, kKindDown);
-      else if (q < n_work) w = make_int4(kKindFin, q - n_up - n_down, 0, 0);
+      else if (q < n_work) {
+        const int f = q - n_up - n_down;
+        w = split_fin ? make_int4(kKindFin, f / kSplit, f % kSplit, 0) : make_int4(kKindFin, f, 0, 0);
+      }
       else w = make_int4(kKindEnd, 0, 0, 0);
       bool ok = true;
       if (lane == 0) {
@@ -645,7 +690,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int4 w = make_int4(epi_item[0], epi_item[1], epi_item[2], epi_item[3]);
       if (w.x == kKindEnd) break;
       if (w.x == kKindFin) {
-        // ---- finalize token t, in the order of the finalize kernel the separate launches use
+        // ---- finalize: a slice of token t (up to 64 tokens) or all of it,
+        // in the reduction order of the finalize kernel the separate launches
+        // use for this many tokens
         const int t = w.y;
         if (et == 0) {
           const bool ready = wait_count(down_done, static_cast<unsigned>(n_down + 1), abort_flag);
@@ -657,20 +704,97 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_sync();
         if (!*epi_go) break;
+        if (et < K) fin_w[et] = ld_cg_f32(args.topk_w + static_cast<size_t>(t) * K + et);
+        epi_sync();
         const int npk = H / 8;
         const uint16_t* xt = args.x + static_cast<size_t>(t) * H;
         const uint16_t* yt = args.y + static_cast<size_t>(t) * K * H;
+        if (split_fin) {
+          // Slice w.z of 8: pack slice*per + et (the few-token kernel's CTA
+          // `slice` of the token's cluster).  Its sum of squares goes to the
+          // workspace; the 8 partials are added in slice order by every slice.
+          const int slice = w.z;
+          const int per = (npk + kSplit - 1) / kSplit;
+          const int p = slice * per + et;
+          const bool live = et < per && p < npk;
+          float a[8];
+          if (live) {
+            unpack8(__ldg(reinterpret_cast<const uint4*>(xt + p * 8)), a);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a[j] = 0.0f;
+          }
+          for (int k0 = 0; k0 < K; k0 += 16) {
+            uint4 v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              v[i] = (live && k0 + i < K)
+                         ? __ldcg(reinterpret_cast<const uint4*>(yt + static_cast<size_t>(k0 + i) * H + p * 8))
+                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (k0 + i >= K) break;
+              const float wk = fin_w[k0 + i];
+              float f[8];
+              unpack8(v[i], f);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) a[j] = fmaf(wk, f[j], a[j]);
+            }
+          }
+          float ss = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = fmaf(a[j], a[j], ss);
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          if (lane == 0) part[et >> 5] = ss;
+          epi_sync();
+          if (et == 0) {
+            float c = 0.0f;
+#pragma unroll
+            for (int wq = 0; wq < 4; ++wq) c += part[wq];
+            fin_part[t * kSplit + slice] = c;
+            __threadfence();
+            red_release_add(fin_cnt + t, 1u);
+            const bool all = wait_count(fin_cnt + t, kSplit, abort_flag);
+            float total = 0.0f;
+            if (all) {
+#pragma unroll
+              for (int r = 0; r < kSplit; ++r) total += ld_cg_f32(fin_part + t * kSplit + r);
+            } else {
+              *abort_flag = 1;
+              set_error(args.err, kErrTimeout);
+            }
+            *fin_total = total;
+            *epi_go = all ? 1 : 0;
+          }
+          epi_sync();
+          if (!*epi_go) break;
+          const float inv = 1.0f / sqrtf(*fin_total / static_cast<float>(H) + args.eps);
+          if (live) {
+            float g[8];
+            unpack8(__ldg(reinterpret_cast<const uint4*>(args.gamma + p * 8)), g);
+            uint4 o;
+            o.x = pack_bf16x2(a[0] * inv * g[0], a[1] * inv * g[1]);
+            o.y = pack_bf16x2(a[2] * inv * g[2], a[3] * inv * g[3]);
+            o.z = pack_bf16x2(a[4] * inv * g[4], a[5] * inv * g[5]);
+            o.w = pack_bf16x2(a[6] * inv * g[6], a[7] * inv * g[7]);
+            *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(t) * H + p * 8) = o;
+            if (args.residual_out != nullptr) {
+              uint4 r;
+              r.x = pack_bf16x2(a[0], a[1]);
+              r.y = pack_bf16x2(a[2], a[3]);
+              r.z = pack_bf16x2(a[4], a[5]);
+              r.w = pack_bf16x2(a[6], a[7]);
+              *reinterpret_cast<uint4*>(args.residual_out + static_cast<size_t>(t) * H + p * 8) = r;
+            }
+          }
+          if (et == 0) mbar_arrive_one(fin_bar);
+          continue;
+        }
+        // The whole token: the many-token kernel's 256-thread CTA, virtual
+        // thread et + 128*(q/4) owning packs vt + 256*(q%4).
         float acc[kSplit][8];
-        // Pack of accumulator set q: up to 64 tokens, the few-token finalize's
-        // order (8 slices of `per` packs, pack q*per + et); more tokens, the
-        // many-token finalize's (a 256-thread CTA: virtual thread et + 128*(q/4)
-        // owns packs vt + 256*(q%4)).
-        const bool split = M <= 64;
-        const int per = (npk + kSplit - 1) / kSplit;
-        auto pack_of = [&](int q) -> int {
-          if (split) return et < per ? q * per + et : npk;
-          return et + 128 * (q >> 2) + 256 * (q & 3);
-        };
+        auto pack_of = [&](int q) -> int { return et + 128 * (q >> 2) + 256 * (q & 3); };
 #pragma unroll
         for (int q = 0; q < kSplit; ++q) {
           const int p = pack_of(q);
@@ -681,8 +805,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i) acc[q][i] = 0.0f;
           }
         }
-        if (et < K) fin_w[et] = ld_cg_f32(args.topk_w + static_cast<size_t>(t) * K + et);
-        epi_sync();
         // 4 expert rows x 8 packs = 32 loads in flight a thread; each element
         // still takes its K terms in increasing k
         for (int k0 = 0; k0 < K; k0 += 4) {
@@ -709,45 +831,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        float total = 0.0f;
-        if (split) {
-          // per slice: the sum of squares over its 128 threads (butterfly, then
-          // the 4 warps in order); the slices added in order
+        // per virtual thread: its packs in order; butterfly per virtual warp;
+        // the 8 virtual warps in order
 #pragma unroll
-          for (int q = 0; q < kSplit; ++q) {
-            float ss = 0.0f;
+        for (int hv = 0; hv < 2; ++hv) {
+          float ss = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) ss = fmaf(acc[q][i], acc[q][i], ss);
+          for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            if (lane == 0) part[q * 4 + (et >> 5)] = ss;
-          }
-          epi_sync();
+            for (int j = 0; j < 8; ++j) ss = fmaf(acc[4 * hv + i][j], acc[4 * hv + i][j], ss);
 #pragma unroll
-          for (int q = 0; q < kSplit; ++q) {
-            float c = 0.0f;
-#pragma unroll
-            for (int wq = 0; wq < 4; ++wq) c += part[q * 4 + wq];
-            total += c;
-          }
-        } else {
-          // per virtual thread: its packs in order; butterfly per virtual warp;
-          // the 8 virtual warps in order
-#pragma unroll
-          for (int hv = 0; hv < 2; ++hv) {
-            float ss = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-              for (int j = 0; j < 8; ++j) ss = fmaf(acc[4 * hv + i][j], acc[4 * hv + i][j], ss);
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            if (lane == 0) part[4 * hv + (et >> 5)] = ss;
-          }
-          epi_sync();
-#pragma unroll
-          for (int wq = 0; wq < 8; ++wq) total += part[wq];
+          for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          if (lane == 0) part[4 * hv + (et >> 5)] = ss;
         }
+        epi_sync();
+        float total = 0.0f;
+#pragma unroll
+        for (int wq = 0; wq < 8; ++wq) total += part[wq];
         epi_sync();  // part[] may be reused by the next item
         const float inv = 1.0f / sqrtf(total / static_cast<float>(H) + args.eps);
 #pragma unroll
