@@ -67,6 +67,9 @@ def parse_args(argv=None):
                    help="override E (a smaller copy of the workload, e.g. for profiler captures)")
     p.add_argument("--tokens", type=int, default=0, help="override M (with --experts: a smaller copy)")
     p.add_argument("--topk", type=int, default=0, help="override top_k (with --experts)")
+    p.add_argument("--route-only", action="store_true",
+                   help="time moe_route alone on the workload's router inputs (no expert weights allocated; "
+                        "a small target for profiler captures of the router kernels)")
     return p.parse_args(argv)
 
 
@@ -538,10 +541,37 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_route_only(args):
+    """moe_route (logits + top-k) on the workload's x, W_r and bias: device time per call and the rate of
+    the logits' fma (M*E*H per call).  A kernel measurement, not a layer number."""
+    import torch
+    import prefill_sigmoid_top_b200 as moe
+    from prefill_sigmoid_top_b200 import inputs
+    cfg = workload(args)
+    w_router, bias, _, x = inputs.router_inputs(cfg)
+    x, w_router, bias = x.cuda(), w_router.cuda(), bias.cuda()
+    for _ in range(max(3, args.warmup)):
+        moe.route(x, w_router, bias, cfg.K)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        moe.route(x, w_router, bias, cfg.K)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    fma = float(cfg.M) * cfg.E * cfg.H
+    print(json.dumps({"kernel": "moe_route", "workload": cfg.name, "M": cfg.M, "E": cfg.E, "H": cfg.H,
+                      "top_k": cfg.K, "us_per_call": us, "fma_per_s": fma / (us * 1e-6),
+                      "steps": args.steps}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.route_only:
+        run_route_only(args)
     else:
         run_ours(args)
 
