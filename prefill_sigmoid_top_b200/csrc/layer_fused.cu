@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kTopkPerLane; ++i) {
         const int e = lane + 32 * i;
         live[u][i] = e < E && tt[u] < M;
-        v[u][i] = live[u][i] ? ld_cg_f32(args.logits + static_cast<size_t>(tt[u]) * E + e) : -INFINITY;
+        // plain L2 loads (not volatile), so that all of them are in flight at once
+        v[u][i] = live[u][i] ? __ldcg(args.logits + static_cast<size_t>(tt[u]) * E + e) : -INFINITY;
       }
     float sel_v[2] = {0.0f, 0.0f};
     int sel_id[2] = {0, 0};
@@ -758,8 +759,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool all = wait_count(fin_cnt + t, kSplit, abort_flag);
             float total = 0.0f;
             if (all) {
+              float pr[kSplit];  // all 8 loads in flight, then added in slice order
 #pragma unroll
-              for (int r = 0; r < kSplit; ++r) total += ld_cg_f32(fin_part + t * kSplit + r);
+              for (int r = 0; r < kSplit; ++r) pr[r] = __ldcg(fin_part + t * kSplit + r);
+#pragma unroll
+              for (int r = 0; r < kSplit; ++r) total += pr[r];
             } else {
               *abort_flag = 1;
               set_error(args.err, kErrTimeout);
