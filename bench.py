@@ -36,9 +36,9 @@ NCU_TRAFFIC = {
     # (workload, kernel): (DRAM bytes per launch, hash of the kernel's sources)
     # decode M=8, the staged up kernel: E=32 capture (1.8243 GB for 31 touched experts) scaled to 95
     (1, "up"): (5_590_700_000, "bf42fabd738f6afa"),
-    # decode M=8, the single-launch layer: E=32 capture (2.7370 GB read + write for 31 touched
-    # experts, 1.0021 x its 2.7312 GB of algorithmic bytes) scaled to 95 touched experts
-    (1, "layer_fused"): (8_387_700_000, "f79e7079afa5b31c"),
+    # decode M=8, the single-launch layer: E=32 capture (2.7368 GB read + write for 31 touched
+    # experts, 1.0020 x its 2.7312 GB of algorithmic bytes) scaled to 95 touched experts
+    (1, "layer_fused"): (8_386_900_000, "d815c00a1de4a117"),
 }
 KERNEL_SOURCES = {
     "up": ["prefill_sigmoid_top_b200/csrc/gemm_bf16.cu", "prefill_sigmoid_top_b200/csrc/common.cuh"],
