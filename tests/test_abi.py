@@ -54,6 +54,21 @@ def test_sizes():
     assert lay["total"] - lay["y"] >= 8 * 16 * 7168 * 2
 
 
+@pytest.mark.parametrize("shape", [C0, C1, moe.Shape(M=64, H=512, I=256, E=256, top_k=16, block_size=16),
+                                   moe.Shape(M=200, H=512, I=256, E=64, top_k=4, block_size=16)],
+                         ids=["C0", "C1", "M64_E256", "M200"])
+def test_single_launch_counters_in_the_cleared_region(shape):
+    """The single-launch layer's counters (grid barrier, work counter, finalize count, one up count per
+    expert, and per token a slice count and 8 partial sums when M <= 64) sit after the error word and
+    before the logits: the region moe_layer clears with one memset before every call."""
+    lay = moe.layer_workspace_layout(shape)
+    words = 3 + shape.E + (9 * shape.M if shape.M <= 64 else 0)
+    assert lay["err_flag"] == 0
+    assert lay["err_flag"] + 4 <= lay["sync"]
+    assert lay["sync"] % 16 == 0
+    assert lay["sync"] + 4 * words <= lay["logits"]
+
+
 @pytest.mark.parametrize("bad", [
     dict(H=255), dict(H=8448), dict(I=64), dict(E=0), dict(E=1025), dict(top_k=0), dict(top_k=9),
     dict(block_size=24), dict(block_size=8), dict(block_size=512), dict(M=0),
