@@ -241,7 +241,9 @@ MOE_API moe_status_t moe_finalize_rmsnorm(const moe_bf16_t* x, const moe_bf16_t*
  * 위한 NKI 레이어 메가커널"), bit-identical to the separate entry points;
  * MOE_FUSED_LAYER=0 in the environment selects the 5-launch form instead, in
  * which the align step runs inside the up projection
- * (moe_grouped_up_swiglu_routed).
+ * (moe_grouped_up_swiglu_routed); moe_layer also takes it by itself when the
+ * single launch cannot be made (a GPU shared with other work that cannot
+ * hold one CTA per SM at once).
  * Intermediates live in ws (moe_layer_workspace_size bytes, 256-byte aligned);
  * the first int32 of ws is the layer's device error word (cleared by each
  * call; read it with moe_get_device_error((const int32_t*)ws, ...)).

@@ -330,7 +330,14 @@ moe_status_t run_layer_fused(const moe_bf16_t* x, const moe_bf16_t* w_router, co
   a.residual_out = residual_out;
   a.err = reinterpret_cast<int32_t*>(base + L.err_flag);
   a.sync = reinterpret_cast<unsigned*>(base + L.sync);
-  return cuda_status(moe::launch_layer_fused(mg, mu, md, mx, mh, a, num_sms(), stream));
+  const cudaError_t e = moe::launch_layer_fused(mg, mu, md, mx, mh, a, num_sms(), stream);
+  if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorInvalidConfiguration || e == cudaErrorInvalidValue) {
+    // nothing was launched (e.g. the GPU is shared and cannot hold one CTA per SM at once): the caller
+    // runs the separate launches instead
+    (void)cudaGetLastError();
+    return MOE_ERR_UNSUPPORTED;
+  }
+  return cuda_status(e);
 }
 
 moe_status_t run_up_routed(const moe_bf16_t* x, const moe_weights_t* w, const int32_t* topk_ids,
@@ -720,8 +727,10 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
 
   // the error word and the single-launch layer's counters, in one region
   if ((st = cuda_status(cudaMemsetAsync(err, 0, L.logits - L.err_flag, cs))) != MOE_OK) return st;
-  if (want_fused_layer(s, w->dtype))
-    return run_layer_fused(x, w_router, bias, w, gamma, eps, s, out, residual_out, ids, tw, base, L, cs);
+  if (want_fused_layer(s, w->dtype)) {
+    st = run_layer_fused(x, w_router, bias, w, gamma, eps, s, out, residual_out, ids, tw, base, L, cs);
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
   float* logits = reinterpret_cast<float*>(base + L.logits);
   if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
     return st;
