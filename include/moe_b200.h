@@ -234,7 +234,7 @@ MOE_API moe_status_t moe_finalize_rmsnorm(const moe_bf16_t* x, const moe_bf16_t*
  * (flashinfer PR #6511 analysis, §6 route chain), with the same results as
  * calling those entry points in turn.  On decode shapes (MOE_W_BF16, at most
  * 24 routed rows per expert on average, M*top_k <= MOE_ROUTED_UP_MAX_SLOTS,
- * E <= 256) the layer is ONE cooperative launch (one CTA pair per SM: the
+ * E <= 256) the layer is ONE cooperative launch (one 192-thread CTA per SM: the
  * router, a grid barrier, the plan, the up and down tiles handed out by a
  * device-side counter with the down tiles of an expert waiting for its up
  * tiles, then the finalize; the megakernel of "AWS Trainium2에서 GLM-5.3-Flash를
@@ -309,8 +309,10 @@ MOE_API size_t moe_nvfp4_blob_bytes(moe_shape_t s, int which);
  *    without launching anything.
  *  - The array is a fixed 4 MiB device allocation made when the library is
  *    loaded; every GPU the process uses holds one until the process exits.
- *  - The first call on each device looks up the array's device address on
- *    that device (the current device at the time of the call); that first
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, which allocates nothing), so the address stays
+ *    right after a device reset or a new primary context.  The first call
+ *    on a device may load the library's device code there, so that first
  *    call should come before any stream capture on the device.
  *  - All calls share the one array: calls whose kernels may overlap on the
  *    GPU (other streams, other host threads) race and give wrong results, so

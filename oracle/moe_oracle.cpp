@@ -223,6 +223,11 @@ void oracle_router_logits(const uint16_t* x, const uint16_t* w_router, const flo
     }
 }
 
+// Non-finite logits are outside the pages' workloads; a NaN logit is read as
+// -inf, so it ranks below every other logit (its expert is picked only when
+// nothing else is left) and its sigmoid score is 0.
+static float key_of(float z) { return std::isnan(z) ? -INFINITY : z; }
+
 // Sigmoid top-k selection and renormalisation for each token.
 // Selection key: the fp32 logit z (sigmoid is monotone, so this is the
 // order of the sigmoid scores; keeping z avoids depending on how exp is
@@ -233,10 +238,11 @@ void oracle_router_logits(const uint16_t* x, const uint16_t* w_router, const flo
 void oracle_topk(const float* z32, int M, int E, int K, int32_t* topk_ids, double* topk_w) {
 #pragma omp parallel for schedule(static)
   for (int t = 0; t < M; ++t) {
-    const float* z = z32 + static_cast<size_t>(t) * E;
+    std::vector<float> z(E);
+    for (int e = 0; e < E; ++e) z[e] = key_of(z32[static_cast<size_t>(t) * E + e]);
     std::vector<int> order(E);
     for (int e = 0; e < E; ++e) order[e] = e;
-    std::sort(order.begin(), order.end(), [z](int a, int b) {
+    std::sort(order.begin(), order.end(), [&z](int a, int b) {
       if (z[a] > z[b]) return true;
       if (z[a] < z[b]) return false;
       return a < b;
@@ -270,7 +276,8 @@ void oracle_topk_ex(const float* z32, const float* sel_bias, int M, int E, int K
   std::vector<double> unused(static_cast<size_t>(M) * K);
   oracle_topk(key.data(), M, E, K, topk_ids, unused.data());
   for (int t = 0; t < M; ++t) {
-    const float* z = z32 + static_cast<size_t>(t) * E;
+    std::vector<float> z(E);
+    for (int e = 0; e < E; ++e) z[e] = key_of(z32[static_cast<size_t>(t) * E + e]);
     double p[64];
     double denom_all = 0.0, zmax = -INFINITY;
     if (scoring == 0) {

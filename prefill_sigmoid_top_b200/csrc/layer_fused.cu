@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int e = lane + 32 * i;
         live[u][i] = e < E && tt[u] < M;
         // plain L2 loads (not volatile), so that all of them are in flight at once
-        v[u][i] = live[u][i] ? __ldcg(args.logits + static_cast<size_t>(tt[u]) * E + e) : -INFINITY;
+        const float z = live[u][i] ? __ldcg(args.logits + static_cast<size_t>(tt[u]) * E + e) : -INFINITY;
+        v[u][i] = isnan(z) ? -INFINITY : z;  // a NaN logit ranks below every other (the router's rule)
       }
     float sel_v[2] = {0.0f, 0.0f};
     int sel_id[2] = {0, 0};

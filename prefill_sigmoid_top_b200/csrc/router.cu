@@ -24,8 +24,6 @@
 //     a routed scale, and a bias that only shifts the selection key.  The
 //     selection is the same warp argmax on the key; the score of a selected
 //     expert is taken from the logit without the selection-only bias.
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "router_dot.cuh"
@@ -170,6 +168,10 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
+// A NaN logit enters the selection (and its score) as -inf: it ranks below
+// every other logit, so a selected id always lies in [0, E).
+__device__ __forceinline__ float selection_key(float z) { return isnan(z) ? -INFINITY : z; }
+
 template <int kPerLane>
 __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restrict__ logits, int M, int E, int K,
                                                           int32_t* __restrict__ topk_ids,
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restric
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
     live[i] = e < E;
-    v[i] = live[i] ? logits[static_cast<size_t>(t) * E + e] : -INFINITY;
+    v[i] = live[i] ? selection_key(logits[static_cast<size_t>(t) * E + e]) : -INFINITY;
   }
   float sel_v = 0.0f;
   int sel_id = 0;
@@ -239,8 +241,8 @@ __global__ void __launch_bounds__(128) router_topk_ext_kernel(const float* __res
   for (int i = 0; i < kPerLane; ++i) {
     const int e = lane + 32 * i;
     live[i] = e < E;
-    z[i] = live[i] ? zt[e] : -INFINITY;
-    v[i] = (live[i] && sel_bias != nullptr) ? __fadd_rn(z[i], sel_bias[e]) : z[i];
+    z[i] = live[i] ? selection_key(zt[e]) : -INFINITY;
+    v[i] = (live[i] && sel_bias != nullptr) ? selection_key(__fadd_rn(z[i], sel_bias[e])) : z[i];
   }
   // softmax over all E experts: max, then the sum of exp(z - max)
   float zmax = -INFINITY, denom = 0.0f;
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(128) router_topk_ext_kernel(const float* __res
   }
   float p = 0.0f;
   if (lane < K) {
-    const float zs = zt[sel_id];
+    const float zs = selection_key(zt[sel_id]);
     if (scoring == MOE_SCORE_SOFTMAX)  // the common 1/denom cancels when renormalising
       p = renormalize ? expf(zs - zmax) : expf(zs - zmax) / denom;
     else
@@ -339,30 +341,20 @@ cudaError_t launch_router_topk_ext(const float* logits, const float* sel_bias, i
 // moe_route_noalloc: moe_route for callers that cannot allocate device memory.
 // The [M,E] logits live in this fixed array instead of a caller workspace.
 // Device code could name the array directly; host code only has a host-side
-// stand-in for it, so the device address is looked up once per device (with
-// that device current) and passed to the kernels as a plain pointer.
+// stand-in for it, so every call looks up the array's device address on the
+// current device and passes it to the kernels as a plain pointer.  The lookup
+// allocates nothing and is not cached: an address kept from an earlier call
+// would dangle after a device reset or a new primary context.
 namespace {
 
 static __device__ __align__(256) float g_route_logits_scratch[MOE_ROUTE_NOALLOC_MAX_LOGITS];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-float* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the array on the current device (set-up on first use).
+// Device address of the array on the current device.
 cudaError_t route_scratch_address(float** out) {
-  int dev = 0;
-  cudaError_t st = cudaGetDevice(&dev);
+  void* ptr = nullptr;
+  const cudaError_t st = cudaGetSymbolAddress(&ptr, g_route_logits_scratch);
   if (st != cudaSuccess) return st;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    st = cudaGetSymbolAddress(&ptr, g_route_logits_scratch);
-    if (st != cudaSuccess) return st;
-    g_scratch_ptr[dev] = static_cast<float*>(ptr);
-  }
-  *out = g_scratch_ptr[dev];
+  *out = static_cast<float*>(ptr);
   return cudaSuccess;
 }
 

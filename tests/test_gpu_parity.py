@@ -90,6 +90,25 @@ def test_router_ties_exact():
     assert torch.allclose(w.cpu(), torch.full((M, K), 1.0 / K), atol=1e-7)
 
 
+def test_router_nan_logits_keep_ids_in_range():
+    # NaN logits (a NaN router row, a NaN token) rank below every other logit, as in the oracle:
+    # ids bit-exact, every id inside [0, E), weights equal where the oracle's are finite.
+    M, H, E, K = 9, 512, 64, 8
+    cfg = inputs.WORKLOADS[0].with_(M=M, H=H, E=E, K=K, bias="normal", seed=41)
+    w_r, b, _, x = inputs.router_inputs(cfg)
+    w_r[[5, 17, 40]] = float("nan")
+    x[4] = float("nan")
+    for route_fn in (moe.route, lambda *a: moe.route_ex(*a)):
+        ids, w = route_fn(x.to(DEV), w_r.to(DEV), b.to(DEV), K)
+        ids_o, w_o = oracle.route(bf16_bits(x), bf16_bits(w_r), b.numpy(), K)
+        ids, w = ids.cpu().numpy(), w.cpu().numpy()
+        assert np.array_equal(ids, ids_o)
+        assert ((ids >= 0) & (ids < E)).all()
+        fin = np.isfinite(w_o)
+        assert np.array_equal(np.isfinite(w), fin)
+        assert np.abs(w[fin] - w_o[fin]).max() <= 1e-6
+
+
 @pytest.mark.parametrize("cid", [1, 2, 3, 4])
 def test_router_bitexact_full_size(cid):
     cfg = inputs.WORKLOADS[cid]

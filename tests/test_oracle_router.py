@@ -109,6 +109,33 @@ def test_topk_ties_and_signed_zero():
     assert np.allclose(w[1], 0.2, rtol=0, atol=1e-15)
 
 
+def test_topk_nan_logit_ranks_last():
+    # A NaN logit (outside the workloads) is read as -inf: the selection is numpy's stable
+    # lexicographic order on (key descending, id ascending) with NaN keys replaced by -inf,
+    # and a NaN expert gets sigmoid weight 0; every id stays inside [0, E).
+    rng = np.random.default_rng(17)
+    z = rng.standard_normal((6, 40)).astype(np.float32)
+    z[0, [3, 9, 30]] = np.nan
+    z[1, :] = np.nan                  # a whole token of NaN: every key -inf, ids 0..K-1
+    z[2, 5] = -np.inf
+    z[2, 6] = np.nan                  # ties with the -inf at 5; 5 < 6 wins
+    z[3, :37] = np.nan                # only 3 finite keys for K = 8
+    K = 8
+    ids, w = oracle.topk(z, K)
+    key = np.where(np.isnan(z), -np.inf, z)
+    for t in range(z.shape[0]):
+        order = np.lexsort((np.arange(z.shape[1]), -key[t].astype(np.float64)))
+        assert ids[t].tolist() == order[:K].tolist()
+    assert ((ids >= 0) & (ids < z.shape[1])).all()
+    assert not (ids[0][:, None] == np.array([3, 9, 30])[None, :]).any()
+    assert ids[1].tolist() == list(range(K))
+    assert np.isnan(w[1]).all()       # 0 / 0: every selected score is 0
+    assert set(ids[3][:3].tolist()) == {37, 38, 39}
+    assert (w[3][3:] == 0).all() and np.allclose(w[3][:3].sum(), 1.0, rtol=0, atol=1e-12)
+    ids_ex, w_ex = oracle.topk_ex(z, K, oracle.SCORING_SIGMOID)
+    assert np.array_equal(ids_ex, ids)
+
+
 def test_weights_sum_order_and_ratio():
     rng = np.random.default_rng(5)
     z = (rng.standard_normal((64, 256)) * 2).astype(np.float32)
