@@ -1,13 +1,22 @@
 #!/usr/bin/env python3
 """Benchmark of the routed-MoE layer on B200 (one JSON line on rank 0).
 
-Default workload: decode, M=8 tokens (H=7168, I=2048, E=256, top_k=16, block 16,
-seed 1).  One step = one pass of the whole layer: route -> align -> up+SwiGLU
--> down -> finalize+RMSNorm, inputs resident in HBM.  The expert weights are
-22.5 GB and each step streams the touched experts' weights (several GB), far
-more than the 126 MB L2, so no L2 flush is needed between steps.
+The metric is the layer's µs and tokens/s at the decode, batch and prefill
+token counts, as a fraction of the roofline that bounds each.  The default run
+measures four workloads back to back (H=7168, I=2048, E=256, top_k=16):
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+  decode_m8           M=8,    block 16, seed 1   (the headline: ``value`` and the top-level keys)
+  batch_m512          M=512,  block 64, seed 2
+  prefill_m2048_zipf  M=2048, block 128, seed 3, Zipf-skewed expert popularity
+  nvfp4_m1000         M=1000, block 16, seed 4, NVFP4 expert weights
+
+and reports every one of them under ``workloads``.  One step = one pass of the
+whole layer (route -> align -> up+SwiGLU -> down -> finalize+RMSNorm) through
+``moe_layer``, inputs resident in HBM.  Each step streams GBs of expert weights,
+far more than the 126 MB L2, so no L2 flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--workloads all|C,C,..]
+                  [--impl ours|reference]
 
 Multi-GPU: the layer is run as independent replicas, one per rank (no
 collective on the data path); rank 0 prints the max-over-ranks time.
@@ -28,14 +37,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-# ncu DRAM traffic of the dominant kernel, per launch, measured on the decode
-# workload (a capture on its E=32 copy, scaled by the touched experts).  Valid
-# only while the kernel sources hash to the recorded value; otherwise "traffic"
-# is reported as null.
+METRIC = "MoE layer tokens/s (decode/batch/prefill routed-MoE layer, H=7168 I=2048 E=256 top_k=16)"
+DEFAULT_WORKLOADS = (1, 2, 3, 4)
+
+# ncu DRAM traffic of a workload's dominant kernel, per launch, from a capture
+# on a smaller copy of the workload scaled to the full one.  Valid only while
+# the kernel sources hash to the recorded value; otherwise "traffic" is null.
 NCU_TRAFFIC = {
     # (workload, kernel): (DRAM bytes per launch, hash of the kernel's sources)
-    # decode M=8, the staged up kernel: E=32 capture (1.8243 GB for 31 touched experts) scaled to 95
-    (1, "up"): (5_590_700_000, "bf42fabd738f6afa"),
     # decode M=8, the single-launch layer: E=32 capture (2.7368 GB read + write for 31 touched
     # experts, 1.0020 x its 2.7312 GB of algorithmic bytes) scaled to 95 touched experts
     (1, "layer_fused"): (8_386_900_000, "d815c00a1de4a117"),
@@ -60,9 +69,13 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--config", type=int, default=1)
+    p.add_argument("--config", type=int, default=1, help="the headline workload (value, top-level keys)")
+    p.add_argument("--workloads", default="default",
+                   help="workloads measured after the headline: 'default' (all four when the headline is the "
+                        "decode workload and no size is overridden, else none), 'all', 'none' or a list like 2,3")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time per workload's CPU baseline")
     p.add_argument("--experts", type=int, default=0,
                    help="override E (a smaller copy of the workload, e.g. for profiler captures)")
     p.add_argument("--tokens", type=int, default=0, help="override M (with --experts: a smaller copy)")
@@ -73,9 +86,9 @@ def parse_args(argv=None):
     return p.parse_args(argv)
 
 
-def workload(args):
+def workload(args, cid=None):
     from prefill_sigmoid_top_b200 import inputs
-    cfg = inputs.WORKLOADS[args.config]
+    cfg = inputs.WORKLOADS[args.config if cid is None else cid]
     if args.experts:
         cfg = cfg.with_(E=args.experts, name=f"{cfg.name}_E{args.experts}")
     if args.tokens:
@@ -83,6 +96,21 @@ def workload(args):
     if args.topk:
         cfg = cfg.with_(K=args.topk, name=f"{cfg.name}_K{args.topk}")
     return cfg
+
+
+def workload_list(args):
+    """The workload ids one run measures, headline first."""
+    overridden = bool(args.experts or args.tokens or args.topk)
+    w = args.workloads
+    if w == "default":
+        rest = list(DEFAULT_WORKLOADS) if (args.config == 1 and not overridden) else []
+    elif w == "all":
+        rest = list(DEFAULT_WORKLOADS)
+    elif w == "none":
+        rest = []
+    else:
+        rest = [int(v) for v in w.split(",") if v.strip()]
+    return [args.config] + [c for c in rest if c != args.config]
 
 
 # ------------------------------------------------------------------ ranks
@@ -186,6 +214,11 @@ def algorithmic_bytes(cfg, touched: int, nvfp4: bool = False):
                 finalize=cfg.M * cfg.K * cfg.H * 2 + 2 * cfg.M * cfg.H * 2)
 
 
+def layer_flops(cfg) -> float:
+    """Dense-equivalent flops of the expert projections: 2 * (gate + up + down) * H * I per routed slot."""
+    return 2.0 * 3 * cfg.H * cfg.I * cfg.M * cfg.K
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -195,29 +228,126 @@ def peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def tensor_peak(bf16_tflops: float, nvfp4: bool) -> float:
+    """Dense tensor peak for the workload's MMA type: the measured bf16 peak, times the nominal
+    fp4 / bf16 ratio (9 / 2.25 PFLOP/s) for NVFP4 weights and activations."""
+    return bf16_tflops * (4.0 if nvfp4 else 1.0)
+
+
+def layer_bound(cfg) -> str:
+    """The roofline a workload is graded against: the tensor pipe for the compute-shaped prefill
+    workload (its target is stated as a fraction of the dense bf16 tensor peak), HBM for the
+    weight-streaming ones.  Both fractions are always reported."""
+    return "tensor" if (cfg.wdtype == "bf16" and cfg.M * cfg.K / cfg.E >= 96) else "hbm"
+
+
+def layer_roofline(cfg, touched, seconds, hbm_peak, tc_peak_bf16, read_ceiling=None):
+    nvfp4 = cfg.wdtype == "nvfp4"
+    ab = algorithmic_bytes(cfg, touched, nvfp4)["layer"]
+    gbs = ab / seconds / 1e9
+    tflops = layer_flops(cfg) / seconds / 1e12
+    tpk = tensor_peak(tc_peak_bf16, nvfp4)
+    r = {"algorithmic_bytes": ab, "GBps": gbs, "frac_hbm": gbs / hbm_peak, "hbm_peak_gbs": hbm_peak,
+         "tflops": tflops, "frac_tensor": tflops / tpk, "tensor_peak_tflops": tpk,
+         "tensor_dtype": "fp4 (measured bf16 x 4)" if nvfp4 else "bf16"}
+    if read_ceiling:
+        r["read_ceiling_gbs"] = read_ceiling
+        r["frac_read_ceiling"] = gbs / read_ceiling
+    bound = layer_bound(cfg)
+    r["bound"] = bound
+    r["frac"] = r["frac_tensor"] if bound == "tensor" else r["frac_hbm"]
+    return r
+
+
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
-    import numpy as np
+def measure_read_ceiling(moe, torch, buf, reps=5):
+    """Device-timed streaming read (moe_measure_hbm_read) of buf: the best GB/s of reps reads."""
+    sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    for _ in range(2):
+        moe.measure_hbm_read(buf, sink)
+    torch.cuda.synchronize()
+    best = 0.0
+    stream = torch.cuda.current_stream()
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moe.measure_hbm_read(buf, sink)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = max(best, buf.numel() * buf.element_size() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    return best
+
+
+def e2e_overlapped(torch, layer_step, x_src, out_shape, steps, warmup):
+    """End-to-end device time of `steps` layer calls whose inputs come from pinned host memory and whose
+    outputs go back to it, every step: x is copied in on one stream, the layer runs on the current stream,
+    out is copied back on a third, with two buffers each, so step k+1's upload and step k-1's download run
+    under step k's layer.  Returns (seconds, the last step's host output, bytes in, bytes out per step)."""
+    comp = torch.cuda.current_stream()
+    up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
+    x_host = x_src.cpu().pin_memory()
+    x_dev = [torch.empty_like(x_src) for _ in range(2)]
+    out_dev = [torch.empty(out_shape, dtype=torch.bfloat16, device=x_src.device) for _ in range(2)]
+    out_host = [torch.empty(out_shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+
+    def run(n):
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_done = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        up_s.wait_stream(comp)
+        down_s.wait_stream(comp)
+        t0.record(up_s)
+        for k in range(n):
+            b = k % 2
+            with torch.cuda.stream(up_s):
+                if k >= 2:
+                    up_s.wait_event(ev_done[k - 2])   # layer k-2 has read x_dev[b]
+                x_dev[b].copy_(x_host, non_blocking=True)
+                ev_in[k].record(up_s)
+            comp.wait_event(ev_in[k])
+            if k >= 2:
+                comp.wait_event(ev_out[k - 2])        # out_dev[b] has been read back
+            layer_step(x_dev[b], out_dev[b])
+            ev_done[k].record(comp)
+            with torch.cuda.stream(down_s):
+                down_s.wait_event(ev_done[k])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                ev_out[k].record(down_s)
+        t1.record(down_s)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) * 1e-3
+
+    run(max(3, warmup))
+    secs = run(steps)
+    last = out_host[(steps - 1) % 2].clone()
+    return secs, last, x_src.numel() * x_src.element_size(), last.numel() * last.element_size()
+
+
+def measure_workload(cfg, args, dev, world, rank, want_cpu, read_ceiling_box):
+    """Times one workload; returns its result dict (see the module docstring)."""
     import torch
 
     import prefill_sigmoid_top_b200 as moe
     from prefill_sigmoid_top_b200 import inputs
 
-    rank, local_rank, world = dist_env()
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    moe.library()  # fail loudly if the CUDA library cannot be loaded
-
-    cfg = workload(args)
     nvfp4 = cfg.wdtype == "nvfp4"
     d = inputs.make_inputs(cfg, dev)
     shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
     stream = torch.cuda.current_stream()
+
+    # the HBM read ceiling, measured once per run on the first workload's weights (8 GB of them)
+    if read_ceiling_box.get("gbs") is None and d["w_gate"].numel() * 2 >= (4 << 30):
+        flat = d["w_gate"].view(-1)
+        read_ceiling_box["gbs"] = measure_read_ceiling(moe, torch, flat[: min(flat.numel(), 4 << 30)])
+        read_ceiling_box["how"] = ("moe_measure_hbm_read: streaming 16-byte non-caching loads of 8 GB of this "
+                                   "run's expert weights, 4 CTAs x 512 threads per SM, best of 5 (CUDA events)")
+
+    # the oracle's inputs for the CPU baseline, taken before the bf16 weights can be dropped (NVFP4)
+    cpu_inputs = None
+    if want_cpu:
+        cpu_inputs = oracle_sample_inputs(cfg, d, n=4 if nvfp4 else min(cfg.M, 8))
+
     nw = None
     if nvfp4:  # weight preparation (quantise + repack) happens once, before any timing
         nw = moe.nvfp4_weights(d["w_gate"], d["w_up"], d["w_down"], shape)
@@ -225,7 +355,7 @@ def run_ours(args):
         del d["w_gate"], d["w_up"], d["w_down"]
         torch.cuda.empty_cache()
 
-    # buffers of the staged pass (the same kernels moe_layer launches)
+    # ---- staged pass: the separate entry points in turn, per-stage events
     route_ws = torch.empty(moe.route_workspace_size(shape), dtype=torch.uint8, device=dev)
     ids = torch.empty(cfg.M, cfg.K, dtype=torch.int32, device=dev)
     tw = torch.empty(cfg.M, cfg.K, dtype=torch.float32, device=dev)
@@ -244,7 +374,6 @@ def run_ours(args):
     h = torch.empty(cap, cfg.I, dtype=torch.bfloat16, device=dev)
     y = torch.empty(cfg.M * cfg.K, cfg.H, dtype=torch.bfloat16, device=dev)
     out = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16, device=dev)
-
     stages = ["route", "align", "up", "down", "finalize"]
 
     def step(evs=None):
@@ -273,13 +402,13 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
     if moe.get_device_error(err) != 0:
-        raise SystemExit("device error during warm-up")
+        raise SystemExit(f"device error during warm-up ({cfg.name})")
     touched = int((plan["expert_counts"] > 0).sum().item())
 
     # Workloads whose weights fit in L2 a few times over get L2 flushed (a 256 MB
     # write) before every timed step; the flush is outside the timed work.
-    ab_pre = algorithmic_bytes(cfg, touched, nvfp4)
-    flush_l2 = ab_pre["layer"] < 4 * 126_000_000
+    ab = algorithmic_bytes(cfg, touched, nvfp4)
+    flush_l2 = ab["layer"] < 4 * 126_000_000
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
 
     def flush():
@@ -287,18 +416,15 @@ def run_ours(args):
             flush_buf.zero_()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
     torch.cuda.synchronize()
     for k in range(args.steps):
         flush()
         step(evs[k])
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
     staged_ms = statistics.mean(e[0].elapsed_time(e[5]) for e in evs)
     out_staged = out.clone()  # the staged pass's result, compared with moe_layer's below
     stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, s in enumerate(stages)}
+    del route_ws, up_ws, down_ws, h, y
 
     # ---- the timed layer: moe_layer (the public entry point, one call per step) on resident inputs
     ws = torch.empty(moe.layer_workspace_size(shape, wdt), dtype=torch.uint8, device=dev)
@@ -315,8 +441,9 @@ def run_ours(args):
     for _ in range(max(3, args.warmup)):
         layer_step(d["x"], out_layer)
     torch.cuda.synchronize()
+
     def timed_loop(body):
-        """Device time of args.steps calls of body(): one event pair around all of them, or, when L2 is
+        """Device time (ms) of args.steps calls of body(): one event pair around all of them, or, when L2 is
         flushed before every call, one pair per call (the flush outside) summed."""
         if not flush_l2:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -343,6 +470,7 @@ def run_ours(args):
         t_wall0 = time.perf_counter()
         total_ms = timed_loop(lambda: layer_step(d["x"], out_layer))
         t_wall = time.perf_counter() - t_wall0
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     ms_per_step = total_ms / args.steps
@@ -350,7 +478,7 @@ def run_ours(args):
     value = aggregate(cfg.M * args.steps, max_s, world)
     eo = moe.layer_workspace_layout(shape, wdt)["err_flag"]
     if moe.get_device_error(ws[eo:eo + 4].view(torch.int32)) != 0:
-        raise SystemExit("device error in the timed layer calls")
+        raise SystemExit(f"device error in the timed layer calls ({cfg.name})")
 
     # ---- the same call replayed from a CUDA graph (launch work taken off the host)
     graph_ms = None
@@ -369,93 +497,140 @@ def run_ours(args):
         graph_ms = timed_loop(graph.replay) / args.steps
         del graph
 
-    # ---- end to end through the public entry point (moe_layer) with host buffers
-    x_host = d["x"].cpu().pin_memory()
-    out_host = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(d["x"])
-
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        layer_step(x_dev, out)
-        out_host.copy_(out, non_blocking=True)
-
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
-    torch.cuda.synchronize()
+    # ---- end to end through the public entry point (moe_layer) with host buffers, copies overlapped
     if world > 1:
         torch.distributed.barrier()
-    e2e_s = reduce_max(timed_loop(e2e_step) / 1e3, world, dev)
+    e2e_s, out_host, h2d_b, d2h_b = e2e_overlapped(torch, layer_step, d["x"], (cfg.M, cfg.H), args.steps,
+                                                   args.warmup)
+    e2e_s = reduce_max(e2e_s, world, dev)
     e2e_value = aggregate(cfg.M * args.steps, e2e_s, world)
     # the e2e output (host), the timed layer's output and the staged pass's output are the same bits
     same = bool(torch.equal(out_host, out_staged.cpu())) and bool(torch.equal(out_layer, out_staged))
 
     hbm_peak, tc_peak, peak_kind = peaks()
-    ab = algorithmic_bytes(cfg, touched, nvfp4)
     up_s = stage_ms["up"] / 1e3
     up_achieved = ab["up"] / up_s / 1e9
-    default_workload = not (args.experts or args.tokens or args.topk)
+    default_size = not (args.experts or args.tokens or args.topk)
+    cid = next((k for k, v in inputs.WORKLOADS.items() if v.name == cfg.name), None)
 
     def ncu_traffic(kernel):
-        tr = NCU_TRAFFIC.get((args.config, kernel)) if default_workload else None
+        tr = NCU_TRAFFIC.get((cid, kernel)) if default_size else None
         return tr[0] if tr is not None and tr[1] == kernel_hash(kernel) else None
 
-    # The dominant kernel: on decode shapes moe_layer is one launch (the whole
-    # layer: its algorithmic bytes over the timed call, which includes the
-    # call's 1 KB memset of its counters); otherwise the up projection of the
-    # staged pass.
+    lroof = layer_roofline(cfg, touched, ms_per_step / 1e3, hbm_peak, tc_peak, read_ceiling_box.get("gbs"))
+    # The dominant kernel: on decode shapes moe_layer is one launch (the whole layer); otherwise the up
+    # projection (the largest share of the staged pass).
     fused = (not nvfp4) and moe.layer_kernel_count(shape, wdt) == 1
     if fused:
-        roof = {"bound": "hbm", "kernel": "layer_fused_kernel (moe_layer: route, plan, up, down, finalize)",
-                "achieved": ab["layer"] / (ms_per_step / 1e3) / 1e9, "algorithmic_bytes": ab["layer"],
-                "traffic": ncu_traffic("layer_fused")}
+        dom = {"kernel": "layer_fused_kernel (moe_layer: route, plan, up, down, finalize)",
+               "achieved": ab["layer"] / (ms_per_step / 1e3) / 1e9, "algorithmic_bytes": ab["layer"],
+               "traffic": ncu_traffic("layer_fused")}
     else:
-        roof = {"bound": "hbm", "kernel": "grouped_up_swiglu", "achieved": up_achieved,
-                "algorithmic_bytes": ab["up"], "traffic": ncu_traffic("up")}
-    roof.update(peak=hbm_peak, unit="GB/s", frac=roof["achieved"] / hbm_peak, peak_source=peak_kind)
-    flops = 2.0 * 3 * cfg.H * cfg.I * cfg.M * cfg.K
-    if nvfp4:
-        tc_peak *= 4.0  # dense fp4 / bf16 nominal ratio (9 / 2.25 PFLOP/s) applied to the measured bf16 peak
+        dom = {"kernel": "grouped_up_swiglu (staged pass)", "achieved": up_achieved,
+               "algorithmic_bytes": ab["up"], "traffic": None}
+    dom.update(bound="hbm", peak=hbm_peak, unit="GB/s", frac=dom["achieved"] / hbm_peak, peak_source=peak_kind)
+    if read_ceiling_box.get("gbs"):
+        dom["read_ceiling_gbs"] = read_ceiling_box["gbs"]
+        dom["frac_read_ceiling"] = dom["achieved"] / read_ceiling_box["gbs"]
+    if dom["frac"] > 1.0:
+        dom["note"] = ("frac > 1: the peak is the pool's measured copy (read + write); a read-only stream runs "
+                       "above it, and frac_read_ceiling compares it with a pure read measured in this run")
 
+    cs = clocks.summary() or {}
+    if cs.get("sm_mhz"):
+        cs["ms_x_mhz"] = ms_per_step * cs["sm_mhz"]  # time x clock: comparable across power-capped runs
+    res = {
+        "workload": cfg.name,
+        "config": {"workload": cfg.name, "M": cfg.M, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.K,
+                   "block_size": cfg.B, "seed": cfg.seed, "router_bias": cfg.bias, "touched_experts": touched,
+                   "weights": cfg.wdtype,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": ("flush: a 256 MB write before every timed step, outside the timed work" if flush_l2 else
+                          "no flush: each step streams GBs of expert weights, far above the 126 MB L2")},
+        "dtype": ("nvfp4 weights+activations (e2m1, e4m3 block-16 scales), fp32 accumulate, bf16 I/O" if nvfp4
+                  else "bf16"),
+        "value": value, "unit": "tokens/s", "ms_per_step": ms_per_step, "us_per_layer": ms_per_step * 1e3,
+        "steps": args.steps,
+        "kernels_us": {s: v * 1e3 for s, v in stage_ms.items()},
+        "staged_us_per_layer": staged_ms * 1e3,
+        "graph_us_per_layer": None if graph_ms is None else graph_ms * 1e3,
+        "gpu_launches_per_step": moe.layer_kernel_count(shape, wdt),
+        "layer_roofline": lroof,
+        "dominant_kernel": dom,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b,
+                "entry_point": "moe_layer",
+                "copies": "x in from pinned host memory and out back to it every step, on two copy streams "
+                          "(double-buffered) under the layer of the neighbouring steps",
+                "matches_staged": same},
+        "clocks": cs,
+        "wall_s_timed": t_wall,
+    }
+    del ws, out_layer, d, nw
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if cpu_inputs is not None:
+        res["cpu_baseline"] = cpu_baseline(cfg, cpu_inputs, target_s=args.cpu_seconds)
+    return res
+
+
+def run_ours(args):
+    import torch
+
+    import prefill_sigmoid_top_b200 as moe
+
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    moe.library()  # fail loudly if the CUDA library cannot be loaded
+
+    ids = workload_list(args)
+    read_ceiling = {}
+    results = []
+    for cid in ids:
+        cfg = workload(args, cid)
+        want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+        results.append(measure_workload(cfg, args, dev, world, rank, want_cpu, read_ceiling))
+    head = results[0]
+
+    hbm_peak, tc_peak, peak_kind = peaks()
+    dom = head["dominant_kernel"]
     result = {
-        "metric": "MoE layer tokens/s (decode/batch/prefill routed-MoE layer, H=7168 I=2048 E=256 top_k=16)",
-        "value": value,
+        "metric": METRIC,
+        "value": head["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": max(3, args.warmup),
-        "ms_per_step": ms_per_step,
-        "us_per_layer": ms_per_step * 1e3,
+        "ms_per_step": head["ms_per_step"],
+        "us_per_layer": head["us_per_layer"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "nvfp4 weights+activations (e2m1, e4m3 block-16 scales), fp32 accumulate, bf16 I/O" if nvfp4 else "bf16",
+        "dtype": head["dtype"],
         "data": "synthetic (seeded; random-init weights of the workload's shapes)",
-        "config": {"workload": cfg.name, "M": cfg.M, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.K,
-                   "block_size": cfg.B, "seed": cfg.seed, "router_bias": cfg.bias, "touched_experts": touched,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": ("flush: a 256 MB write before every timed step, outside the timed work" if flush_l2 else
-                          "no flush: each step streams GBs of expert weights, far above the 126 MB L2")},
-        "kernels_us": {s: v * 1e3 for s, v in stage_ms.items()},
-        "staged_us_per_layer": staged_ms * 1e3,
-        "graph_us_per_layer": None if graph_ms is None else graph_ms * 1e3,
-        "gpu_launches": moe.layer_kernel_count(shape, wdt) * args.steps,
-        "roofline": {k: roof[k] for k in ("bound", "kernel", "achieved", "peak", "unit", "frac", "traffic",
-                                          "algorithmic_bytes", "peak_source")},
-        "staged_up_roofline": {"achieved": up_achieved, "frac": up_achieved / hbm_peak, "traffic": ncu_traffic("up"),
-                               "algorithmic_bytes": ab["up"]},
-        "layer_roofline": {"algorithmic_bytes": ab["layer"], "GBps": ab["layer"] / (ms_per_step / 1e3) / 1e9,
-                           "frac_hbm": ab["layer"] / (ms_per_step / 1e3) / 1e9 / hbm_peak,
-                           "tflops": flops / (ms_per_step / 1e3) / 1e12,
-                           "frac_bf16_tensor": flops / (ms_per_step / 1e3) / 1e12 / tc_peak},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": cfg.M * cfg.H * 2,
-                "d2h_bytes_per_step": cfg.M * cfg.H * 2, "entry_point": "moe_layer", "matches_staged": same},
-        "wall_s_timed": t_wall,
+        "config": head["config"],
+        "kernels_us": head["kernels_us"],
+        "staged_us_per_layer": head["staged_us_per_layer"],
+        "graph_us_per_layer": head["graph_us_per_layer"],
+        "gpu_launches": head["gpu_launches_per_step"] * args.steps,
+        "roofline": {k: dom[k] for k in ("bound", "kernel", "achieved", "peak", "unit", "frac", "traffic",
+                                         "algorithmic_bytes", "peak_source", "read_ceiling_gbs",
+                                         "frac_read_ceiling", "note") if k in dom},
+        "layer_roofline": head["layer_roofline"],
+        "e2e": head["e2e"],
+        "clocks": head["clocks"],
+        "peaks": {"hbm_copy_gbs": hbm_peak, "bf16_tflops": tc_peak, "source": peak_kind,
+                  "hbm_read_ceiling_gbs": read_ceiling.get("gbs"), "hbm_read_ceiling_how": read_ceiling.get("how")},
+        "workloads": {r["workload"]: {k: v for k, v in r.items() if k != "workload"} for r in results},
+        "wall_s_timed": sum(r["wall_s_timed"] for r in results),
     }
-    cs = clocks.summary()
-    if cs is not None:
-        result["clocks"] = cs
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not nvfp4:
-        result["cpu_baseline"] = cpu_baseline(cfg, d, target_s=12.0)
+    if "cpu_baseline" in head:
+        result["cpu_baseline"] = head["cpu_baseline"]
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -463,37 +638,44 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------------ oracle timing
-def _oracle_host_inputs(cfg, d):
-    import numpy as np
+def oracle_sample_inputs(cfg, d, n):
+    """Host inputs of the oracle for the first n tokens of the workload: x, router, gamma, and the weights
+    of the experts those tokens route to (bf16 bits; for NVFP4 workloads quantised by the oracle itself)."""
     import oracle
     from prefill_sigmoid_top_b200.inputs import bf16_bits
-    x, wr, b, g = bf16_bits(d["x"]), bf16_bits(d["w_router"]), d["bias"].cpu().numpy(), bf16_bits(d["gamma"])
+    x, wr, b, g = (bf16_bits(d["x"][:n]), bf16_bits(d["w_router"]), d["bias"].cpu().numpy(),
+                   bf16_bits(d["gamma"]))
     ids, _ = oracle.route(x, wr, b, cfg.K)
     need = sorted(set(int(e) for e in ids.ravel()))
     wg, wu, wd = [None] * cfg.E, [None] * cfg.E, [None] * cfg.E
     for e in need:
         wg[e], wu[e], wd[e] = bf16_bits(d["w_gate"][e]), bf16_bits(d["w_up"][e]), bf16_bits(d["w_down"][e])
-    return x, wr, b, g, wg, wu, wd
+        if cfg.wdtype == "nvfp4":
+            wg[e], wu[e], wd[e] = (oracle.nvfp4_quantize_bf16(wg[e]), oracle.nvfp4_quantize_bf16(wu[e]),
+                                   oracle.nvfp4_quantize_bf16(wd[e]))
+    return dict(x=x, wr=wr, b=b, g=g, wg=wg, wu=wu, wd=wd, n=n, experts=len(need))
 
 
-def cpu_baseline(cfg, d, target_s=12.0, max_tokens=None):
-    """Times the CPU oracle (as it stands) on a bounded sample of the same workload."""
-    import numpy as np
+def cpu_baseline(cfg, ci, target_s=10.0):
+    """Times the CPU oracle (as it stands) on a bounded sample of the workload: the first n tokens, as one
+    layer call, repeated until target_s seconds have passed."""
     import oracle
-    x, wr, b, g, wg, wu, wd = _oracle_host_inputs(cfg, d)
-    n = cfg.M if max_tokens is None else min(cfg.M, max_tokens)
-    tokens_done, t0 = 0, time.perf_counter()
+    n = ci["n"]
+    t0 = time.perf_counter()
     reps = 0
     while True:
-        oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=np.arange(n, dtype=np.int32))
-        tokens_done += n
+        if cfg.wdtype == "nvfp4":
+            oracle.layer_nvfp4(ci["x"], ci["wr"], ci["b"], ci["wg"], ci["wu"], ci["wd"], ci["g"], cfg.eps, cfg.K)
+        else:
+            oracle.layer(ci["x"], ci["wr"], ci["b"], ci["wg"], ci["wu"], ci["wd"], ci["g"], cfg.eps, cfg.K)
         reps += 1
         if time.perf_counter() - t0 >= target_s:
             break
     el = time.perf_counter() - t0
-    return {"value": tokens_done / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{reps} x full layer on {n} of {cfg.M} tokens of {cfg.name} (fp64 C++ oracle, OpenMP), "
-                      f"{el:.1f} s"}
+    kind = "NVFP4 layer" if cfg.wdtype == "nvfp4" else "layer"
+    return {"value": n * reps / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} x the {kind} on the first {n} of {cfg.M} tokens of {cfg.name} as one call "
+                      f"({ci['experts']} experts; fp64 C++ oracle, OpenMP), {el:.1f} s"}
 
 
 def run_reference(args):
@@ -507,33 +689,39 @@ def run_reference(args):
     cfg = workload(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     d = inputs.make_inputs(cfg, dev)
-    x, wr, b, g, wg, wu, wd = _oracle_host_inputs(cfg, d)
+    ci = oracle_sample_inputs(cfg, d, cfg.M if cfg.wdtype == "bf16" else min(cfg.M, 8))
     del d
-    touched = int(len(set(int(e) for e in oracle.route(x, wr, b, cfg.K)[0].ravel())))
+    touched = ci["experts"]
+
+    def call(n):  # the layer on the first n tokens (NVFP4: those tokens as one call)
+        if cfg.wdtype == "nvfp4":
+            oracle.layer_nvfp4(ci["x"][:n], ci["wr"], ci["b"], ci["wg"], ci["wu"], ci["wd"], ci["g"], cfg.eps, cfg.K)
+        else:
+            oracle.layer(ci["x"], ci["wr"], ci["b"], ci["wg"], ci["wu"], ci["wd"], ci["g"], cfg.eps, cfg.K,
+                         tokens=np.arange(n, dtype=np.int32))
+
     # size one step so that the whole run stays within a few minutes
     t0 = time.perf_counter()
-    oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=np.arange(1, dtype=np.int32))
+    call(1)
     per_token = time.perf_counter() - t0
     budget_per_step = 120.0 / max(1, args.steps + args.warmup)
-    n = int(max(1, min(cfg.M, budget_per_step // max(per_token, 1e-3))))
-    toks = np.arange(n, dtype=np.int32)
+    n = int(max(1, min(ci["n"], budget_per_step // max(per_token, 1e-3))))
     for _ in range(args.warmup):
-        oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=toks)
+        call(n)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.layer(x, wr, b, wg, wu, wd, g, cfg.eps, cfg.K, tokens=toks)
+        call(n)
     el = time.perf_counter() - t0
     value = n * args.steps / el
     sample = f"{n} of {cfg.M} tokens of {cfg.name} per step (fp64 C++ oracle, OpenMP)"
     print(json.dumps({
-        "impl": "reference", "metric": "MoE layer tokens/s (decode/batch/prefill routed-MoE layer, H=7168 I=2048 "
-                                      "E=256 top_k=16)",
+        "impl": "reference", "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": cfg.name, "M": cfg.M, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.K,
                    "block_size": cfg.B, "seed": cfg.seed, "router_bias": cfg.bias, "touched_experts": touched,
-                   "parallelism": "host cores (CPU oracle)",
+                   "weights": cfg.wdtype, "parallelism": "host cores (CPU oracle)",
                    "l2": "no flush: each step streams GBs of expert weights, far above the 126 MB L2"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},

@@ -114,6 +114,7 @@ def _declare(L):
         "moe_get_device_error": (st, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
         "moe_route_noalloc": (st, [vp, vp, vp, _Shape, vp, vp, vp]),
         "moe_selftest_wait_timeout": (st, [vp, ctypes.c_uint32, vp]),
+        "moe_measure_hbm_read": (st, [vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -454,6 +455,14 @@ def layer_nvfp4(x, w_router, bias, nw: NVFP4Weights, gamma, eps, top_k, block_si
 def selftest_wait_timeout(err_flag, limit_us: int = 1000):
     """Run the kernel whose bounded wait always expires (see moe_selftest_wait_timeout)."""
     _check(library().moe_selftest_wait_timeout(_ptr(err_flag), int(limit_us), _stream()), "moe_selftest_wait_timeout")
+
+
+def measure_hbm_read(buf, sink):
+    """Enqueue one streaming read of the whole tensor ``buf`` (the HBM read-ceiling kernel of
+    moe_measure_hbm_read); ``sink`` is a device int32/uint32 word."""
+    _need_cuda(buf, sink)
+    _check(library().moe_measure_hbm_read(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), _stream()),
+           "moe_measure_hbm_read")
 
 
 def get_device_error(err_flag) -> int:

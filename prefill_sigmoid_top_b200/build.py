@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 SOURCES = ["api.cu", "router.cu", "align.cu", "finalize.cu", "gemm_bf16.cu", "gemm_persistent.cu", "gemm_pair.cu",
-           "nvfp4.cu", "layer_fused.cu"]
+           "nvfp4.cu", "layer_fused.cu", "measure.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-DNDEBUG", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include"), "-I", CSRC]
@@ -28,7 +28,8 @@ def _stale(out: str, deps: list[str]) -> bool:
 def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
-    headers.append(os.path.join(ROOT, "include", "moe_b200.h"))
+    inc = os.path.join(ROOT, "include")
+    headers += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
     flags = FLAGS + (extra_flags or [])
     jobs = []
     objs = []

@@ -74,3 +74,33 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
 def rms(a) -> float:
     a = np.asarray(a, dtype=np.float64)
     return float(np.sqrt(np.mean(a * a)))
+
+
+def sample_tokens(ids_o, n_total, seed, tile):
+    """Tokens checked at full size: every token routed to the coldest touched expert; the first two and
+    all of the last (ragged) `tile`-row token tile of the hottest expert (its slots in ascending slot id,
+    the plan order); then random tokens up to n_total."""
+    M, K = ids_o.shape
+    flat = ids_o.ravel()
+    counts = np.bincount(flat)
+    hot = int(np.argmax(counts))
+    cold = int(np.argmin(np.where(counts > 0, counts, np.iinfo(np.int64).max)))
+    hot_slots = np.nonzero(flat == hot)[0]
+    last_tile = hot_slots[(len(hot_slots) - 1) // tile * tile:]
+    pick = set(int(s) // K for s in hot_slots[:2]) | set(int(s) // K for s in last_tile)
+    pick |= set(int(s) // K for s in np.nonzero(flat == cold)[0])
+    rng = np.random.default_rng(seed)
+    for t in rng.permutation(M):
+        if len(pick) >= n_total:
+            break
+        pick.add(int(t))
+    return np.array(sorted(pick), np.int32)
+
+
+def token_tile(cfg):
+    """Token-tile width of the workload's grouped kernels (2-SM pairs: 256 rows from 96 routed rows per
+    expert on average, else 128; NVFP4: 128; decode shapes: 32)."""
+    per_expert = cfg.M * cfg.K / cfg.E
+    if cfg.wdtype == "nvfp4":
+        return 128
+    return 32 if per_expert <= 24 else (256 if per_expert >= 96 else 128)

@@ -14,13 +14,16 @@ from prefill_sigmoid_top_b200 import _Plan, _Shape, _Weights, _Layout, _RouteOpt
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+                 if f.endswith(".h"))
 
 FAKE = ctypes.c_void_p(0x10000)       # aligned non-null address, never dereferenced
 FAKE_MIS = ctypes.c_void_p(0x10008)   # 8-byte aligned only
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    """Every function that a header under include/ declares."""
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, re.M)))
 
 

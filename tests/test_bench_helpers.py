@@ -90,3 +90,28 @@ def test_command_line_defaults(bench):
     assert a.config == 3 and a.route_only and a.steps == 5
     w = bench.workload(bench.parse_args(["--config", "1", "--experts", "32"]))
     assert (w.M, w.E, w.K) == (8, 32, 16) and w.name == "decode_m8_E32"
+
+
+def test_default_run_measures_all_four_workloads(bench):
+    assert bench.workload_list(bench.parse_args([])) == [1, 2, 3, 4]
+    assert bench.workload_list(bench.parse_args(["--config", "3"])) == [3]
+    assert bench.workload_list(bench.parse_args(["--experts", "32"])) == [1]  # a smaller copy: headline only
+    assert bench.workload_list(bench.parse_args(["--config", "0", "--workloads", "all"])) == [0, 1, 2, 3, 4]
+    assert bench.workload_list(bench.parse_args(["--workloads", "none"])) == [1]
+
+
+def test_layer_roofline_fractions(bench):
+    # prefill: 2 * 3 * H * I * M * K flops; graded on the bf16 tensor peak, HBM fraction beside it
+    cfg = inputs.WORKLOADS[3]
+    r = bench.layer_roofline(cfg, 256, 0.004, 6541.5, 1617.9, read_ceiling=7200.0)
+    flops = 2 * 3 * 7168 * 2048 * 2048 * 16
+    assert r["tflops"] == pytest.approx(flops / 0.004 / 1e12)
+    assert r["bound"] == "tensor" and r["frac"] == r["frac_tensor"] == pytest.approx(r["tflops"] / 1617.9)
+    ab = 256 * 88_080_384 + 256 * 7168 * 2 + 2 * 2048 * 7168 * 2
+    assert r["algorithmic_bytes"] == ab and r["frac_hbm"] == pytest.approx(ab / 0.004 / 1e9 / 6541.5)
+    assert r["frac_read_ceiling"] == pytest.approx(ab / 0.004 / 1e9 / 7200.0)
+    # NVFP4: HBM-graded; the tensor peak is the measured bf16 peak x 4 (nominal fp4 / bf16)
+    r4 = bench.layer_roofline(inputs.WORKLOADS[4], 256, 0.0015, 6541.5, 1617.9)
+    assert r4["bound"] == "hbm" and r4["tensor_peak_tflops"] == pytest.approx(4 * 1617.9)
+    assert bench.layer_roofline(inputs.WORKLOADS[1], 95, 0.0012, 6541.5, 1617.9)["bound"] == "hbm"
+    assert bench.layer_roofline(inputs.WORKLOADS[2], 256, 0.0036, 6541.5, 1617.9)["bound"] == "hbm"

@@ -16,7 +16,7 @@ import torch
 import oracle
 import prefill_sigmoid_top_b200 as moe
 from prefill_sigmoid_top_b200 import inputs
-from tests._util import bf16_bits, bits_to_f64, rms
+from tests._util import bf16_bits, bits_to_f64, rms, sample_tokens, token_tile
 
 pytestmark = pytest.mark.gpu
 
@@ -348,18 +348,6 @@ def test_layer_small(cfg):
     assert np.abs(bits_to_f64(g["res"]) - rref).max() <= 2e-2 * rms(rref)
 
 
-def _sample_tokens(ids_o, n_random, seed):
-    """Tokens routed to the busiest expert (first and last) plus random ones."""
-    M, K = ids_o.shape
-    counts = np.bincount(ids_o.ravel(), minlength=int(ids_o.max()) + 1)
-    hot = int(np.argmax(counts))
-    on_hot = np.nonzero((ids_o == hot).any(axis=1))[0]
-    rng = np.random.default_rng(seed)
-    pick = {int(on_hot[0]), int(on_hot[-1])} | set(int(t) for t in rng.choice(M, size=min(M, n_random),
-                                                                               replace=False))
-    return np.array(sorted(pick), np.int32)
-
-
 @pytest.mark.slow
 @pytest.mark.parametrize("cid", [1, 2, 3])
 def test_layer_full_size_sampled(cid):
@@ -370,7 +358,8 @@ def test_layer_full_size_sampled(cid):
     ids_o, w_o = oracle.route(hb["x"], hb["w_router"], hb["bias"], cfg.K)
     assert np.array_equal(g["ids"], ids_o)
     assert np.abs(g["w"] - w_o).max() <= 1e-6
-    tokens = np.arange(cfg.M, dtype=np.int32) if cfg.M <= 8 else _sample_tokens(ids_o, 3, cid)
+    tokens = np.arange(cfg.M, dtype=np.int32) if cfg.M <= 32 else sample_tokens(ids_o, 32, cid, token_tile(cfg))
+    assert len(tokens) >= min(cfg.M, 32)
     wg, wu, wd = expert_lists(d, ids_o[tokens].ravel(), cfg.E)
     r = oracle.layer(hb["x"], hb["w_router"], hb["bias"], wg, wu, wd, hb["gamma"], cfg.eps, cfg.K, tokens=tokens)
     ref = r["out_f64"]
