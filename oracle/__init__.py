@@ -69,6 +69,11 @@ def lib():
                 "oracle_layer_nvfp4": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32,
                                              i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
                 "oracle_num_threads": (i32, []),
+                "oracle_tp_partial": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
+                                            vp, vp]),
+                "oracle_rmsnorm_rows": (None, [vp, vp, f64, i32, i32, vp, vp, vp]),
+                "oracle_layer_tp": (i32, [vp, vp, vp, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, vp, i32, vp, vp,
+                                          vp, vp, vp, vp, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -337,3 +342,67 @@ def layer_nvfp4(x, w_router, bias, gate_q, up_q, down_q, gamma, eps, K, tokens=N
         raise RuntimeError(f"oracle_layer_nvfp4 status {st}")
     return dict(ids_all=ids, w_all=w, h_all=h, y=y, out=out, residual=res, out_f64=o64, residual_f64=s64,
                 tokens=tok)
+
+
+# ------------------------------------------------------------------ tensor parallel
+def _tp_common(x, w_router, gamma, w_gate, w_up, w_down, tokens):
+    x, w_router = _u16(x), _u16(w_router)
+    M, H = x.shape
+    E = w_router.shape[0]
+    wg = [None if a is None else _u16(a) for a in w_gate]
+    wu = [None if a is None else _u16(a) for a in w_up]
+    wd = [None if a is None else _u16(a) for a in w_down]
+    I = next(a for a in wg if a is not None).shape[0]
+    tok = np.arange(M, dtype=np.int32) if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    return x, w_router, wg, wu, wd, M, H, E, I, tok
+
+
+def tp_partial(x, w_router, bias, w_gate, w_up, w_down, K, G, rank, tokens=None, want_y=False):
+    """One rank's part of the tensor-parallel layer (I split over G ranks): returns dict(ids, w,
+    p [n,H] fp64 = (rank 0: x) + sum_k w_k y_r[k], y [n,K,H] bf16 bits of the rank's partial rows if asked)."""
+    x, w_router, wg, wu, wd, M, H, E, I, tok = _tp_common(x, w_router, None, w_gate, w_up, w_down, tokens)
+    n = len(tok)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    ids = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float64)
+    p = np.empty((n, H), np.float64)
+    y = np.empty((n, K, H), np.uint16) if want_y else None
+    st = lib().oracle_tp_partial(_p(x), _p(w_router), _p(b), _ptr_table(wg), _ptr_table(wu), _ptr_table(wd), H, I, E,
+                                 K, G, rank, _p(tok), n, _p(ids), _p(w), _p(p), _p(y))
+    if st != 0:
+        raise RuntimeError(f"oracle_tp_partial status {st}")
+    return dict(ids=ids, w=w, p=p, y=y, tokens=tok)
+
+
+def rmsnorm_rows(s, gamma, eps):
+    """s [n,H] fp64 -> (out bf16 bits, residual bf16 bits, out before rounding fp64)."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    n, H = s.shape
+    out = np.empty((n, H), np.uint16)
+    res = np.empty((n, H), np.uint16)
+    o64 = np.empty((n, H), np.float64)
+    lib().oracle_rmsnorm_rows(_p(s), _p(_u16(gamma)), float(eps), n, H, _p(out), _p(res), _p(o64))
+    return out, res, o64
+
+
+def layer_tp(x, w_router, bias, w_gate, w_up, w_down, gamma, eps, K, G, tokens=None, want_y_parts=False):
+    """The tensor-parallel layer on G ranks (every rank's part computed here): dict(ids, w, out, residual,
+    out_f64, residual_f64, y_parts [G,n,K,H] bf16 bits if asked)."""
+    x, w_router, wg, wu, wd, M, H, E, I, tok = _tp_common(x, w_router, gamma, w_gate, w_up, w_down, tokens)
+    gamma = _u16(gamma)
+    n = len(tok)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    ids = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float64)
+    yp = np.empty((G, n, K, H), np.uint16) if want_y_parts else None
+    out = np.empty((n, H), np.uint16)
+    res = np.empty((n, H), np.uint16)
+    o64 = np.empty((n, H), np.float64)
+    s64 = np.empty((n, H), np.float64)
+    st = lib().oracle_layer_tp(_p(x), _p(w_router), _p(b), _ptr_table(wg), _ptr_table(wu), _ptr_table(wd), _p(gamma),
+                               float(eps), H, I, E, K, G, _p(tok), n, _p(ids), _p(w), _p(yp), _p(out), _p(res), _p(o64),
+                               _p(s64))
+    if st != 0:
+        raise RuntimeError(f"oracle_layer_tp status {st}")
+    return dict(ids=ids, w=w, out=out, residual=res, out_f64=o64, residual_f64=s64, y_parts=yp, tokens=tok)
+

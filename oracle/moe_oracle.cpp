@@ -679,6 +679,111 @@ int oracle_layer_nvfp4(const uint16_t* x, const uint16_t* w_router, const float*
   return 0;
 }
 
+// ------------------------------------------------------------ tensor parallel
+// The layer with the expert intermediate dimension I split over G ranks, and
+// the finalize fused with the reduction across the ranks and the RMSNorm
+// (flashinfer PR #5701 analysis, intro: "MoE finalize + All-Reduce +
+// RMSNorm").  Reading: rank r holds rows [r*I/G, (r+1)*I/G) of W_gate[e] and
+// W_up[e] and the same columns of W_down[e]; its h is that slice of the
+// unsharded h (each h column depends on its own rows only), and its partial
+// down projection is rounded once to bf16, the rank's stored intermediate:
+//   y_r[t,k,c] = bf16( sum_{i in slice r} h[t,k,i] * W_down[e][c,i] )   (fp64 sum)
+//   p_r[t,c]   = (r == 0 ? x[t,c] : 0) + sum_k w[t,k] * y_r[t,k,c]      (fp64, k in order)
+// The residual enters once (on rank 0), so for G = 1 p_0 is exactly the
+// finalize's s.  Per chosen token i: p_out[i*H..] (fp64), y_out[(i*K+k)*H..]
+// (bf16, nullable), ids/w as oracle_layer.  Returns oracle_layer's codes.
+int oracle_tp_partial(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                      const uint16_t* const* w_gate, const uint16_t* const* w_up, const uint16_t* const* w_down,
+                      int H, int I, int E, int K, int G, int rank, const int32_t* tokens, int n_tokens,
+                      int32_t* topk_ids, double* topk_w, double* p_out, uint16_t* y_out) {
+  if (G < 1 || rank < 0 || rank >= G || I % G != 0) return 2;
+  const int Ir = I / G, i0 = rank * Ir;
+  std::vector<float> z(static_cast<size_t>(E));
+  for (int i = 0; i < n_tokens; ++i) {
+    const uint16_t* xt = x + static_cast<size_t>(tokens[i]) * H;
+    for (int e = 0; e < E; ++e) z[e] = canonical_logit(xt, w_router + static_cast<size_t>(e) * H, H, bias ? bias[e] : 0.0f);
+    oracle_topk(z.data(), 1, E, K, topk_ids + static_cast<size_t>(i) * K, topk_w + static_cast<size_t>(i) * K);
+    for (int k = 0; k < K; ++k) {
+      const int e = topk_ids[static_cast<size_t>(i) * K + k];
+      if (e < 0 || e >= E) return 4;
+      if (!w_gate[e] || !w_up[e] || !w_down[e]) return 3;
+    }
+  }
+  std::vector<uint16_t> y(static_cast<size_t>(n_tokens) * K * H);
+  const int n_slots = n_tokens * K;
+#pragma omp parallel for schedule(dynamic)
+  for (int sl = 0; sl < n_slots; ++sl) {
+    const int i = sl / K;
+    const int e = topk_ids[sl];
+    const uint16_t* xt = x + static_cast<size_t>(tokens[i]) * H;
+    std::vector<double> hd(Ir);
+    for (int j = 0; j < Ir; ++j) {  // this rank's columns of h, as oracle_expert computes them
+      double g = 0.0, u = 0.0;
+      const uint16_t* wg = w_gate[e] + static_cast<size_t>(i0 + j) * H;
+      const uint16_t* wu = w_up[e] + static_cast<size_t>(i0 + j) * H;
+      for (int c = 0; c < H; ++c) {
+        g += bf16_value(xt[c]) * bf16_value(wg[c]);
+        u += bf16_value(xt[c]) * bf16_value(wu[c]);
+      }
+      hd[j] = bf16_value(bf16_round(g * sigmoid(g) * u));
+    }
+    for (int c = 0; c < H; ++c) {
+      double acc = 0.0;
+      const uint16_t* wd = w_down[e] + static_cast<size_t>(c) * I + i0;
+      for (int j = 0; j < Ir; ++j) acc += hd[j] * bf16_value(wd[j]);
+      y[static_cast<size_t>(sl) * H + c] = bf16_round(acc);
+    }
+  }
+  for (int i = 0; i < n_tokens; ++i)
+    for (int c = 0; c < H; ++c) {
+      double acc = rank == 0 ? bf16_value(x[static_cast<size_t>(tokens[i]) * H + c]) : 0.0;
+      for (int k = 0; k < K; ++k)
+        acc += topk_w[static_cast<size_t>(i) * K + k] * bf16_value(y[(static_cast<size_t>(i) * K + k) * H + c]);
+      p_out[static_cast<size_t>(i) * H + c] = acc;
+    }
+  if (y_out) std::memcpy(y_out, y.data(), y.size() * sizeof(uint16_t));
+  return 0;
+}
+
+// RMSNorm of rows s [n,H] (fp64): out = bf16(s / sqrt(mean_h(s^2) + eps) * gamma),
+// residual_out = bf16(s) (nullable), out64 = out before its rounding (nullable).
+void oracle_rmsnorm_rows(const double* s, const uint16_t* gamma, double eps, int n, int H, uint16_t* out,
+                         uint16_t* residual_out, double* out64) {
+  for (int i = 0; i < n; ++i) {
+    const double* st = s + static_cast<size_t>(i) * H;
+    double ss = 0.0;
+    for (int c = 0; c < H; ++c) ss += st[c] * st[c];
+    const double inv = 1.0 / std::sqrt(ss / H + eps);
+    for (int c = 0; c < H; ++c) {
+      const double o = st[c] * inv * bf16_value(gamma[c]);
+      out[static_cast<size_t>(i) * H + c] = bf16_round(o);
+      if (residual_out) residual_out[static_cast<size_t>(i) * H + c] = bf16_round(st[c]);
+      if (out64) out64[static_cast<size_t>(i) * H + c] = o;
+    }
+  }
+}
+
+// The tensor-parallel layer on G ranks, every rank's part computed here:
+// s = p_0 + p_1 + ... + p_{G-1} (fp64, rank order), then oracle_rmsnorm_rows.
+// y_parts (nullable) receives each rank's partial rows, [G][n][K][H] bf16.
+int oracle_layer_tp(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                    const uint16_t* const* w_gate, const uint16_t* const* w_up, const uint16_t* const* w_down,
+                    const uint16_t* gamma, float eps, int H, int I, int E, int K, int G, const int32_t* tokens,
+                    int n_tokens, int32_t* topk_ids, double* topk_w, uint16_t* y_parts, uint16_t* out,
+                    uint16_t* residual_out, double* out64, double* s64) {
+  std::vector<double> s(static_cast<size_t>(n_tokens) * H, 0.0), p(static_cast<size_t>(n_tokens) * H);
+  for (int r = 0; r < G; ++r) {
+    const int st = oracle_tp_partial(x, w_router, bias, w_gate, w_up, w_down, H, I, E, K, G, r, tokens, n_tokens,
+                                     topk_ids, topk_w, p.data(),
+                                     y_parts ? y_parts + static_cast<size_t>(r) * n_tokens * K * H : nullptr);
+    if (st != 0) return st;
+    for (size_t j = 0; j < s.size(); ++j) s[j] = r == 0 ? p[j] : s[j] + p[j];
+  }
+  oracle_rmsnorm_rows(s.data(), gamma, static_cast<double>(eps), n_tokens, H, out, residual_out, out64);
+  if (s64) std::memcpy(s64, s.data(), s.size() * sizeof(double));
+  return 0;
+}
+
 int oracle_num_threads() {
 #ifdef _OPENMP
   return omp_get_max_threads();

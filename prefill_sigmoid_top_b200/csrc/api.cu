@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "moe_b200.h"
+#include "moe_b200_tp.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -522,6 +523,60 @@ moe_layer_ws_layout_t layer_layout(const moe_shape_t& s, moe_wdtype_t dt) {
   return L;
 }
 
+moe_status_t check_layer_args(const moe_bf16_t* x, const moe_bf16_t* w_router, const moe_weights_t* w,
+                              const moe_bf16_t* gamma, float eps, const moe_shape_t& s, const moe_bf16_t* out,
+                              const moe_bf16_t* residual_out) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if ((st = check_weights(w, s)) != MOE_OK) return st;
+  if (!x || !w_router || !gamma || !out || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(gamma) || !aligned16(out) || !aligned16(w->gate) ||
+      !aligned16(w->up) || !aligned16(w->down) || (residual_out && !aligned16(residual_out)))
+    return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// Route -> plan -> up -> down of the layer as separate launches, leaving y [M*K, H] in the workspace
+// (the finalize is the caller's: single-GPU or fused with the exchange across ranks).
+moe_status_t run_layer_to_y(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias,
+                            const moe_weights_t* w, const moe_shape_t& s, uint8_t* base,
+                            const moe_layer_ws_layout_t& L, int32_t* ids, float* tw, cudaStream_t cs) {
+  moe_status_t st;
+  auto* err = reinterpret_cast<int32_t*>(base + L.err_flag);
+  auto* sorted = reinterpret_cast<int32_t*>(base + L.sorted_ids);
+  auto* bexp = reinterpret_cast<int32_t*>(base + L.block_expert);
+  auto* counts = reinterpret_cast<int32_t*>(base + L.expert_counts);
+  auto* offs = reinterpret_cast<int32_t*>(base + L.expert_offsets);
+  auto* ntpp = reinterpret_cast<int32_t*>(base + L.num_tokens_post_padded);
+  auto* h = reinterpret_cast<moe_bf16_t*>(base + L.h);
+  auto* y = reinterpret_cast<moe_bf16_t*>(base + L.y);
+  float* logits = reinterpret_cast<float*>(base + L.logits);
+  if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
+    return st;
+  if ((st = cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, ids, tw, cs))) != MOE_OK) return st;
+  moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
+  if (want_self_route(s, w->dtype)) {
+    if ((st = run_up_routed(x, w, ids, s, sorted, bexp, counts, offs, ntpp, h, err, cs)) != MOE_OK) return st;
+    return run_down(h, w, &plan, s, y, err, cs);
+  }
+  if ((st = cuda_status(moe::launch_align(ids, s.M, s.top_k, s.E, s.block_size, sorted, bexp, counts, offs, ntpp,
+                                          err, cs))) != MOE_OK)
+    return st;
+  if (w->dtype == MOE_W_NVFP4) {
+    // max |h| comes out of the up kernel's epilogue into the down activation copy's amax word
+    uint8_t* act = base + L.act_scratch;
+    uint8_t* act_h = act + x_act_layout(s).total;
+    auto* h_amax = reinterpret_cast<unsigned*>(act_h + h_act_layout(s).amax);
+    if ((st = cuda_status(cudaMemsetAsync(h_amax, 0, sizeof(unsigned), cs))) != MOE_OK) return st;
+    if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs, h_amax)) != MOE_OK) return st;
+    return run_down_nvfp4(h, w, &plan, s, y, act_h, err, cs, true);
+  }
+  if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
+  return run_down(h, w, &plan, s, y, err, cs);
+}
+
 }  // namespace
 
 namespace moe {
@@ -701,15 +756,8 @@ moe_status_t moe_layer_workspace_layout(moe_shape_t s, moe_wdtype_t dtype, moe_l
 moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, const moe_weights_t* w,
                        const moe_bf16_t* gamma, float eps, moe_shape_t s, moe_bf16_t* out, moe_bf16_t* residual_out,
                        int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  moe_status_t st = check_shape(s);
+  moe_status_t st = check_layer_args(x, w_router, w, gamma, eps, s, out, residual_out);
   if (st != MOE_OK) return st;
-  if (!w) return MOE_ERR_INVALID_ARG;
-  if ((st = check_weights(w, s)) != MOE_OK) return st;
-  if (!x || !w_router || !gamma || !out || !w->gate || !w->up || !w->down) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w_router) || !aligned16(gamma) || !aligned16(out) || !aligned16(w->gate) ||
-      !aligned16(w->up) || !aligned16(w->down) || (residual_out && !aligned16(residual_out)))
-    return MOE_ERR_INVALID_ARG;
-  if (!(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
   const moe_layer_ws_layout_t L = layer_layout(s, w->dtype);
   if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   auto cs = static_cast<cudaStream_t>(stream);
@@ -717,12 +765,6 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   auto* err = reinterpret_cast<int32_t*>(base + L.err_flag);
   int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + L.topk_ids);
   float* tw = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + L.topk_w);
-  auto* sorted = reinterpret_cast<int32_t*>(base + L.sorted_ids);
-  auto* bexp = reinterpret_cast<int32_t*>(base + L.block_expert);
-  auto* counts = reinterpret_cast<int32_t*>(base + L.expert_counts);
-  auto* offs = reinterpret_cast<int32_t*>(base + L.expert_offsets);
-  auto* ntpp = reinterpret_cast<int32_t*>(base + L.num_tokens_post_padded);
-  auto* h = reinterpret_cast<moe_bf16_t*>(base + L.h);
   auto* y = reinterpret_cast<moe_bf16_t*>(base + L.y);
 
   // the error word and the single-launch layer's counters, in one region
@@ -731,32 +773,41 @@ moe_status_t moe_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
     st = run_layer_fused(x, w_router, bias, w, gamma, eps, s, out, residual_out, ids, tw, base, L, cs);
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
-  float* logits = reinterpret_cast<float*>(base + L.logits);
-  if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
-    return st;
-  if ((st = cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, ids, tw, cs))) != MOE_OK) return st;
-  moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
-  if (want_self_route(s, w->dtype)) {
-    if ((st = run_up_routed(x, w, ids, s, sorted, bexp, counts, offs, ntpp, h, err, cs)) != MOE_OK) return st;
-    if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
-    return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
-  }
-  if ((st = cuda_status(moe::launch_align(ids, s.M, s.top_k, s.E, s.block_size, sorted, bexp, counts, offs, ntpp,
-                                          err, cs))) != MOE_OK)
-    return st;
-  if (w->dtype == MOE_W_NVFP4) {
-    // max |h| comes out of the up kernel's epilogue into the down activation copy's amax word
-    uint8_t* act = base + L.act_scratch;
-    uint8_t* act_h = act + x_act_layout(s).total;
-    auto* h_amax = reinterpret_cast<unsigned*>(act_h + h_act_layout(s).amax);
-    if ((st = cuda_status(cudaMemsetAsync(h_amax, 0, sizeof(unsigned), cs))) != MOE_OK) return st;
-    if ((st = run_up_nvfp4(x, w, &plan, s, h, act, err, cs, h_amax)) != MOE_OK) return st;
-    if ((st = run_down_nvfp4(h, w, &plan, s, y, act_h, err, cs, true)) != MOE_OK) return st;
-  } else {
-    if ((st = run_up(x, w, &plan, s, h, base + L.act_scratch, L.total - L.act_scratch, err, cs)) != MOE_OK) return st;
-    if ((st = run_down(h, w, &plan, s, y, err, cs)) != MOE_OK) return st;
-  }
+  if ((st = run_layer_to_y(x, w_router, bias, w, s, base, L, ids, tw, cs)) != MOE_OK) return st;
   return cuda_status(moe::launch_finalize(x, y, tw, gamma, eps, s.M, s.top_k, s.H, out, residual_out, cs));
+}
+
+size_t moe_tp_layer_workspace_size(moe_shape_t s) { return moe_layer_workspace_size(s, MOE_W_BF16); }
+
+moe_status_t moe_tp_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const float* bias, const moe_weights_t* w,
+                          const moe_bf16_t* gamma, float eps, moe_shape_t s, const moe_tp_group_t* g,
+                          moe_bf16_t* out, moe_bf16_t* residual_out, int32_t* topk_ids_out, float* topk_w_out,
+                          void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_layer_args(x, w_router, w, gamma, eps, s, out, residual_out);
+  if (st != MOE_OK) return st;
+  if (w->dtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+  if (g == nullptr || g->rank < 0 || g->rank >= g->world) return MOE_ERR_INVALID_ARG;
+  if (g->world < 1 || g->world > MOE_TP_MAX_RANKS || s.M > g->max_tokens || s.H != g->hidden)
+    return MOE_ERR_UNSUPPORTED;
+  if (g->world > 1)
+    for (int r = 0; r < g->world; ++r)
+      if (g->bufs[r] == nullptr || (reinterpret_cast<uintptr_t>(g->bufs[r]) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  const moe_layer_ws_layout_t L = layer_layout(s, MOE_W_BF16);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  auto cs = static_cast<cudaStream_t>(stream);
+  auto* base = static_cast<uint8_t*>(ws);
+  auto* err = reinterpret_cast<int32_t*>(base + L.err_flag);
+  int32_t* ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t*>(base + L.topk_ids);
+  float* tw = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + L.topk_w);
+  const auto* y = reinterpret_cast<const uint16_t*>(base + L.y);
+  if ((st = cuda_status(cudaMemsetAsync(err, 0, L.logits - L.err_flag, cs))) != MOE_OK) return st;
+  // this rank's partial expert rows (its slice of I), then the finalize fused with the exchange
+  if ((st = run_layer_to_y(x, w_router, bias, w, s, base, L, ids, tw, cs)) != MOE_OK) return st;
+  const uint16_t* ys[1] = {y};
+  uint16_t* outs[1] = {out};
+  uint16_t* rs[1] = {residual_out};
+  return cuda_status(moe::launch_tp_finalize(x, ys, tw, gamma, eps, s.M, s.top_k, s.H, g->world, g->max_tokens,
+                                             g->rank, 1, g->bufs, outs, rs, err, cs));
 }
 
 int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype) {

@@ -33,6 +33,17 @@ cudaError_t launch_finalize(const uint16_t* x, const uint16_t* y, const float* t
                             float eps, int M, int K, int H, uint16_t* out, uint16_t* residual_out,
                             cudaStream_t stream);
 
+// tp_finalize.cu: the tensor-parallel finalize (reduction across ranks fused with the norm).
+// `rows` CTA rows play ranks rank0 .. rank0 + rows - 1 (1 for a real rank; G when all ranks
+// are emulated on one GPU); ys / outs / residual_outs hold one pointer per row, bufs one
+// group buffer per rank (null when G == 1).
+cudaError_t launch_tp_finalize(const uint16_t* x, const uint16_t* const* ys, const float* topk_w,
+                               const uint16_t* gamma, float eps, int M, int K, int H, int G, int max_tokens,
+                               int rank0, int rows, void* const* bufs, uint16_t* const* outs,
+                               uint16_t* const* residual_outs, int32_t* err, cudaStream_t stream);
+size_t tp_buffer_bytes(int G, int max_tokens, int H);
+int tp_protocol(int M, int G, int max_tokens);
+
 // finalize.cu: one-warp kernel whose bounded wait can never be satisfied.
 cudaError_t launch_wait_timeout_selftest(int32_t* err, uint64_t limit_ns, cudaStream_t stream);
 
