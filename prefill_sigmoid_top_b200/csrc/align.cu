@@ -17,6 +17,9 @@
 //     cursor + (rank among equal experts in the 32-slot group);
 //  D. padding rows get the sentinel M*K; block b gets the expert found by a
 //     binary search for the last prefix[e] <= b*B.
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -158,6 +161,173 @@ __global__ void __launch_bounds__(kWarps * 32) align_kernel(const int32_t* __res
 }
 
 
+// Many slots: C CTAs, CTA c placing the slots of its own contiguous segment
+// [c*seg, (c+1)*seg).  Every CTA reads all the ids (they sit in L2) and counts,
+// per expert, all of them and those before its segment, so each one knows the
+// padded prefix and where its segment's slots of expert e start inside e's
+// rows without exchanging anything with the other CTAs.  Inside the segment
+// the placement is the one-CTA kernel's (per-warp counts, then a stable
+// in-order scatter), so the plan is the same, bit for bit.  CTA c also writes
+// the padding of experts e = c, c + C, ... and the block -> expert entries of
+// blocks b = c, c + C, ...
+template <int kWarps>
+__global__ void __launch_bounds__(kWarps * 32) align_multi_kernel(const int32_t* __restrict__ topk_ids, int n, int E,
+                                                               int B, int seg, int32_t* __restrict__ sorted_ids,
+                                                               int32_t* __restrict__ block_expert,
+                                                               int32_t* __restrict__ counts_out,
+                                                               int32_t* __restrict__ offsets_out,
+                                                               int32_t* __restrict__ ntpp_out, int32_t* err) {
+  constexpr int kThreads = kWarps * 32;
+  extern __shared__ int smem[];
+  int* all = smem;                   // [E] every slot
+  int* before = all + E;             // [E] slots before this CTA's segment
+  int* prefix = before + E;          // [E + 1]
+  int* hist = prefix + E + 1;        // [kWarps][E]: this segment's counts per warp, then write cursors
+  __shared__ int warp_sums[kWarps];
+  __shared__ int bad;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const int c = blockIdx.x, C = gridDim.x;
+  const int s_begin = min(n, c * seg), s_end = min(n, s_begin + seg);
+
+  for (int i = tid; i < 2 * E; i += kThreads) smem[i] = 0;
+  for (int i = tid; i < kWarps * E; i += kThreads) hist[i] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+
+  // counts over all slots and over the slots before the segment
+  for (int f = tid; f < n; f += kThreads) {
+    const int e = __ldg(topk_ids + f);
+    if (e >= 0 && e < E) {
+      atomicAdd(&all[e], 1);
+      if (f < s_begin) atomicAdd(&before[e], 1);
+    } else {
+      bad = 1;
+    }
+  }
+  // this segment, split into one contiguous piece per warp
+  const int wseg = (s_end - s_begin + kWarps - 1) / kWarps;
+  const int f_begin = min(s_end, s_begin + warp * wseg), f_end = min(s_end, f_begin + wseg);
+  for (int base = f_begin; base < f_end; base += 32) {
+    const int f = base + lane;
+    if (f < f_end) {
+      const int e = __ldg(topk_ids + f);
+      if (e >= 0 && e < E) atomicAdd(&hist[warp * E + e], 1);
+    }
+  }
+  __syncthreads();
+  if (bad) {
+    if (tid == 0 && c == 0) set_error(err, kErrInvalidInput);
+    return;
+  }
+
+  // padded exclusive prefix over the experts, one block scan per kThreads experts
+  int carry = 0;
+  for (int e0 = 0; e0 < E; e0 += kThreads) {
+    const int e = e0 + tid;
+    const int padded = e < E ? (all[e] + B - 1) / B * B : 0;
+    int incl = padded;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int ws = lane < kWarps ? warp_sums[lane] : 0;
+      int wincl = ws;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, wincl, off);
+        if (lane >= off) wincl += v;
+      }
+      if (lane < kWarps) warp_sums[lane] = wincl - ws;
+    }
+    __syncthreads();
+    if (e < E) prefix[e] = carry + warp_sums[warp] + incl - padded;
+    __syncthreads();
+    const int last = min(E, e0 + kThreads) - 1;
+    carry = prefix[last] + (all[last] + B - 1) / B * B;
+    __syncthreads();
+  }
+  if (tid == 0) prefix[E] = carry;
+  __syncthreads();  // every prefix[] entry is written before any thread reads it
+
+  const int total = prefix[E];
+  for (int e = tid; e < E; e += kThreads) {
+    if (c == 0) {
+      counts_out[e] = all[e];
+      offsets_out[e] = prefix[e];
+    }
+    int run = prefix[e] + before[e];
+    for (int w = 0; w < kWarps; ++w) {
+      const int cnt = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += cnt;
+    }
+  }
+  if (tid == 0 && c == 0) {
+    offsets_out[E] = total;
+    *ntpp_out = total;
+  }
+  __syncthreads();
+
+  // stable scatter of this segment
+  for (int base = f_begin; base < f_end; base += 32) {
+    const int f = base + lane;
+    const bool act = f < f_end;
+    const int e = act ? __ldg(topk_ids + f) : -1;
+    const unsigned actmask = __ballot_sync(0xffffffffu, act);
+    const unsigned peers = __match_any_sync(0xffffffffu, e) & actmask;
+    int pos = 0;
+    if (act) pos = hist[warp * E + e] + __popc(peers & lt_mask);
+    __syncwarp();
+    if (act) {
+      sorted_ids[pos] = f;
+      if ((__ffs(peers) - 1) == lane) hist[warp * E + e] += __popc(peers);
+    }
+    __syncwarp();
+  }
+
+  // padding of this CTA's experts and block -> expert of its blocks
+  for (int e = c + C * warp; e < E; e += C * kWarps)
+    for (int pos = prefix[e] + all[e] + lane; pos < prefix[e + 1]; pos += 32) sorted_ids[pos] = n;
+  for (int b = c + C * tid; b * B < total; b += C * kThreads) {
+    const int row = b * B;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    block_expert[b] = lo;
+  }
+}
+
+template <int kWarps>
+cudaError_t launch_align_multi(const int32_t* topk_ids, int n, int E, int B, int32_t* sorted_ids,
+                               int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets, int32_t* ntpp,
+                               int32_t* err, cudaStream_t stream) {
+  const size_t smem = sizeof(int) * (3 * static_cast<size_t>(E) + 1 + static_cast<size_t>(kWarps) * E);
+  if (smem > kSmemLimit) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    st = cudaFuncSetAttribute(align_multi_kernel<kWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kSmemLimit));
+    if (st != cudaSuccess) return st;
+    attr_set[dev] = true;
+  }
+  const int seg = 512;
+  const int ctas = (n + seg - 1) / seg;
+  align_multi_kernel<kWarps><<<ctas, kWarps * 32, smem, stream>>>(topk_ids, n, E, B, seg, sorted_ids, block_expert,
+                                                                expert_counts, expert_offsets, ntpp, err);
+  return cudaGetLastError();
+}
+
 template <int kWarps>
 cudaError_t launch_align_variant(const int32_t* topk_ids, int n, int E, int B, int32_t* sorted_ids,
                                  int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets,
@@ -181,15 +351,25 @@ cudaError_t launch_align_variant(const int32_t* topk_ids, int n, int E, int B, i
   return cudaGetLastError();
 }
 
+// MOE_ALIGN_MULTI=0 keeps the one-CTA kernel for every size (the tests compare both).
+bool align_multi_enabled() {
+  const char* env = std::getenv("MOE_ALIGN_MULTI");
+  return env == nullptr || std::strcmp(env, "0") != 0;
+}
+
 }  // namespace
 
-// One CTA; its thread count must cover the experts (one thread per expert in
-// the prefix step).  Few slots: 8 warps, so that the per-expert loops over
-// the warps' histogram rows are short; otherwise 32 warps.
+// Up to 4096 slots: one CTA, whose thread count must cover the experts (one
+// thread per expert in the prefix step); 8 warps, so that the per-expert loops
+// over the warps' histogram rows are short (else 32 warps).  More slots: the
+// multi-CTA kernel, one CTA per 512 slots.
 cudaError_t launch_align(const int32_t* topk_ids, int M, int K, int E, int B, int32_t* sorted_ids,
                          int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets, int32_t* ntpp,
                          int32_t* err, cudaStream_t stream) {
   const int n = M * K;
+  if (n > 4096 && align_multi_enabled())  // many slots: one CTA per 512 of them
+    return launch_align_multi<16>(topk_ids, n, E, B, sorted_ids, block_expert, expert_counts, expert_offsets, ntpp,
+                                  err, stream);
   if (n <= 4096 && E <= 256)
     return launch_align_variant<8>(topk_ids, n, E, B, sorted_ids, block_expert, expert_counts, expert_offsets, ntpp,
                                    err, stream);

@@ -182,6 +182,23 @@ def test_align_invalid_id_sets_error_without_fault(bad):
     _compare_plan(_gpu_plan(ids_ok, 8, 16), oracle.align(ids_ok, 8, 16), 16)
 
 
+@pytest.mark.parametrize("multi", ["1", "0"])
+def test_align_large_one_and_many_ctas(multi, monkeypatch):
+    # more than 4096 slots: the multi-CTA kernel (default) and the one-CTA kernel give the oracle's plan
+    monkeypatch.setenv("MOE_ALIGN_MULTI", multi)
+    rng = np.random.default_rng(91)
+    for M, K, E, B in [(2048, 16, 256, 128), (1000, 16, 256, 16), (600, 13, 1024, 256), (5000, 8, 9, 32),
+                       (4097, 1, 64, 16)]:
+        p = 1.0 / np.arange(1, E + 1) ** 1.1
+        ids = np.stack([rng.choice(E, size=K, replace=False, p=p / p.sum()) for _ in range(M)]).astype(np.int32)
+        _compare_plan(_gpu_plan(ids, E, B), oracle.align(ids, E, B), B)
+    bad = rng.integers(0, 64, size=(700, 8)).astype(np.int32)
+    bad[650, 3] = 64
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    _gpu_plan(bad, 64, 16, err)
+    assert moe.get_device_error(err) == 4
+
+
 def test_align_repeat_stress():
     # many calls on fresh random inputs; every result bit-exact against the oracle
     rng = np.random.default_rng(2024)
