@@ -263,4 +263,41 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// silu(g) * u = g * u / (1 + e^-g) with the hardware exponential and a fast
+// divide: relative error a few 1e-7, far below the bf16 step (2^-8) that the
+// product is rounded to; e^-g = inf (g < -88) gives 0, the limit.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
+
+__device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
+}
+
+// 8 x 8 transpose of 32-bit words inside each group of 8 lanes (b = lane % 8):
+// on entry lane b holds v[i] = A[b][i], on exit v[i] = A[i][b].  Three
+// butterfly stages; each swaps the off-diagonal blocks of size s between
+// lanes b and b ^ s (12 shuffles in all).  The epilogues use it to turn a
+// lane-per-column tile (the tensor-memory layout) into lane-per-row runs of
+// 8 columns, so that each lane writes 16 contiguous bytes.
+__device__ __forceinline__ void transpose8x8(uint32_t (&v)[8], int b) {
+#pragma unroll
+  for (int s = 4; s >= 1; s >>= 1) {
+    const bool hi = (b & s) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i & s) continue;
+      const uint32_t send = hi ? v[i] : v[i | s];
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, s);
+      if (hi)
+        v[i] = recv;
+      else
+        v[i | s] = recv;
+    }
+  }
+}
+
+// Eight bf16 values (low 16 bits of v[0..7]) as one 16-byte vector.
+__device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[8]) {
+  return make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16), v[6] | (v[7] << 16));
+}
+
 }  // namespace moe

@@ -33,8 +33,8 @@
 //   down: weight block w = rows 512w..512w+511 of W_down as two M = 256
 //         halves; CTA r holds rows 512w + 128r.. and 512w + 256 + 128r..;
 //         y[slot, col] = bf16(acc), scattered to the slot.
-// Warp roles (384 threads per CTA): 0 = weight producer, 1 = MMA issuer
-// (leader only), 2 = token-row producer, 3 = idle, 4..11 = epilogue.
+// Warp roles (640 threads per CTA): 0 = weight producer, 1 = MMA issuer
+// (leader only), 2 = token-row producer, 3 = idle, 4..19 = epilogue.
 // All mbarrier waits are bounded; a timeout sets the error word and unwinds,
 // and both CTAs still meet at the final cluster barrier.
 #include "common.cuh"
@@ -48,7 +48,7 @@ constexpr int kBM = 128;                  // weight rows per CTA (MMA M = 256 pe
 constexpr int kBK = 64;                   // contraction elements per stage
 constexpr int kBoxBytes = kBM * kBK * 2;  // one 128 x 64 bf16 box: 16 KB
 constexpr int kBRows = 32;                // rows per token-row box
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;  // four per tensor-memory lane quarter: the drain is latency-bound
 constexpr int kThreads = 128 + 32 * kEpiWarps;
 
 template <int kNmax, int kStagesA, int kStagesB>
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue (both CTAs: their own 128 rows)
     const int q = warp & 3;
-    const int half_c = (warp - 4) >> 2;
+    const int part_c = (warp - 4) >> 2;  // which of the four 16-column chunks of every 64 this warp drains
     int j = 0;
     for (int tile = pair; tile < total; tile += npairs, ++j) {
       const TileCoord c = decode_tile<kNmax>(prefix, cnt, E, tile);
@@ -349,31 +349,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           ids[i] = (n < nrows) ? args.sorted_ids[row0 + n] : -1;
         }
       }
-      auto* out = reinterpret_cast<__nv_bfloat16*>(args.out);
       const int colbase = kUp ? c.w * 2 * kBM + static_cast<int>(rank) * kBM
                               : c.w * 4 * kBM + static_cast<int>(rank) * kBM;
-      for (int cb = 16 * half_c; cb < N; cb += 32) {
+      // lane l holds column col0 + l (its tensor-memory lane) for the tokens of each 16-column chunk;
+      // 8 x 8 transposes inside each group of 8 lanes give lane (8 g + b) token b's columns
+      // col0 + 8 g .. + 7, written as one 16-byte store per 8 tokens
+      const int g8 = lane >> 3, b8 = lane & 7;
+      const int col8 = colbase + q * 32 + 8 * g8;
+      for (int cb = 16 * part_c; cb < N; cb += 64) {
         uint32_t v0[16], v1[16];
         tmem_load_16(lane_base + cb, v0);
         tmem_load_16(lane_base + kNmax + cb, v1);
         tmem_load_wait();
         const int id_word = kUp ? 0 : pick<kNmax / 32>(ids, cb >> 5);
 #pragma unroll
-        for (int qq = 0; qq < 16; ++qq) {
-          const int n = cb + qq;
-          const int col = colbase + q * 32 + lane;
+        for (int m = 0; m < 2; ++m) {
+          const int n = cb + 8 * m + b8;  // the token this lane writes after the transpose
           if (kUp) {
-            if (n < nrows) {
-              const float g = __uint_as_float(v0[qq]);
-              const float u = __uint_as_float(v1[qq]);
-              out[static_cast<size_t>(row0 + n) * args.out_ld + col] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+            uint32_t hv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float g = __uint_as_float(v0[8 * m + i]);
+              const float u = __uint_as_float(v1[8 * m + i]);
+              hv[i] = bf16_bits_rn(silu_mul(g, u));
             }
+            transpose8x8(hv, b8);
+            if (n < nrows)
+              *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(row0 + n) * args.out_ld + col8) =
+                  pack8_bf16(hv);
           } else {
-            const int id = __shfl_sync(0xffffffffu, id_word, (cb & 31) + qq);
+            uint32_t a[8], bb[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              a[i] = bf16_bits_rn(__uint_as_float(v0[8 * m + i]));
+              bb[i] = bf16_bits_rn(__uint_as_float(v1[8 * m + i]));
+            }
+            transpose8x8(a, b8);
+            transpose8x8(bb, b8);
+            const int id = __shfl_sync(0xffffffffu, id_word, (cb & 31) + 8 * m + b8);
             if (n < nrows && id >= 0 && id < nslots) {
-              out[static_cast<size_t>(id) * args.out_ld + col] = __float2bfloat16_rn(__uint_as_float(v0[qq]));
-              out[static_cast<size_t>(id) * args.out_ld + col + 2 * kBM] =
-                  __float2bfloat16_rn(__uint_as_float(v1[qq]));
+              uint16_t* yr = args.out + static_cast<size_t>(id) * args.out_ld + col8;
+              *reinterpret_cast<uint4*>(yr) = pack8_bf16(a);
+              *reinterpret_cast<uint4*>(yr + 2 * kBM) = pack8_bf16(bb);
             }
           }
         }
