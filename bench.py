@@ -80,6 +80,9 @@ def parse_args(argv=None):
                    help="override E (a smaller copy of the workload, e.g. for profiler captures)")
     p.add_argument("--tokens", type=int, default=0, help="override M (with --experts: a smaller copy)")
     p.add_argument("--topk", type=int, default=0, help="override top_k (with --experts)")
+    p.add_argument("--tp-emulate", type=int, default=0,
+                   help="time the tensor-parallel finalize with this many ranks emulated on one GPU (one cooperative "
+                        "launch; partial rows are seeded random bf16 of the workload's shape)")
     p.add_argument("--route-only", action="store_true",
                    help="time moe_route alone on the workload's router inputs (no expert weights allocated; "
                         "a small target for profiler captures of the router kernels)")
@@ -754,10 +757,47 @@ def run_route_only(args):
                       "steps": args.steps}), flush=True)
 
 
+def run_tp_emulated(args):
+    """The tensor-parallel finalize (cross-rank reduction fused with residual + RMSNorm) with G ranks emulated
+    on one GPU: device time per call and the bytes it moves per rank.  A kernel measurement: the exchange goes
+    through this GPU's memory, not NVLink."""
+    import torch
+    import prefill_sigmoid_top_b200 as moe
+    from prefill_sigmoid_top_b200 import inputs, tp
+    cfg = workload(args)
+    G = args.tp_emulate
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed)
+    x = torch.randn(cfg.M, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
+    gamma = torch.ones(cfg.H, dtype=torch.bfloat16, device="cuda")
+    tw = torch.softmax(torch.randn(cfg.M, cfg.K, generator=g, device="cuda"), dim=1)
+    ys = [(0.1 * torch.randn(cfg.M * cfg.K, cfg.H, generator=g, device="cuda")).to(torch.bfloat16) for _ in range(G)]
+    bufs = [torch.zeros(tp.buffer_bytes(G, cfg.M, cfg.H), dtype=torch.uint8, device="cuda") for _ in range(G)]
+    outs = [torch.empty_like(x) for _ in range(G)]
+    for _ in range(max(3, args.warmup)):
+        tp.tp_finalize_emulated(x, ys, tw, gamma, cfg.eps, cfg.M, bufs, outs)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        tp.tp_finalize_emulated(x, ys, tw, gamma, cfg.eps, cfg.M, bufs, outs)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    proto = tp.protocol(cfg.M, G, cfg.M)
+    row = cfg.H * 4
+    sent = (G - 1) * cfg.M * row if proto == "oneshot" else (G - 1) / G * cfg.M * (row + 2 * cfg.H)
+    print(json.dumps({"kernel": "tp_finalize_kernel (emulated ranks, one GPU)", "workload": cfg.name, "ranks": G,
+                      "protocol": proto, "M": cfg.M, "H": cfg.H, "top_k": cfg.K, "us_per_call": us,
+                      "y_bytes_per_rank": cfg.M * cfg.K * cfg.H * 2, "exchange_bytes_sent_per_rank": int(sent),
+                      "steps": args.steps}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.tp_emulate:
+        run_tp_emulated(args)
     elif args.route_only:
         run_route_only(args)
     else:

@@ -25,17 +25,25 @@ def _stale(out: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+TRACE_LIB = os.path.join(PKG, "libmoe_b200_trace.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          trace: bool = False) -> str:
+    """Compile the library; trace=True builds the timeline variant of the 2-SM pair GEMMs instead
+    (-DMOE_PAIR_TRACE, into libmoe_b200_trace.so; see pair_trace.py), never loaded by the package."""
+    build_dir = BUILD + ("_trace" if trace else "")
+    lib = TRACE_LIB if trace else LIB
+    os.makedirs(build_dir, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     inc = os.path.join(ROOT, "include")
     headers += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
-    flags = FLAGS + (extra_flags or [])
+    flags = FLAGS + (["-DMOE_PAIR_TRACE"] if trace else []) + (extra_flags or [])
     jobs = []
     objs = []
     for src in SOURCES:
         path = os.path.join(CSRC, src)
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        obj = os.path.join(build_dir, src.replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, [path, *headers]):
             jobs.append([NVCC, *flags, "-c", path, "-o", obj])
@@ -45,12 +53,12 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
                 sys.stderr.write(res.stdout + res.stderr)
             if res.returncode != 0:
                 raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", tmp])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, trace="--trace" in sys.argv))

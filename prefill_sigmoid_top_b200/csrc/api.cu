@@ -235,6 +235,23 @@ int pair_nmax(const moe_shape_t& s) {
   return per_expert >= 96.0 ? 256 : 128;
 }
 
+// Whether the 2-SM pair up kernel gathers its x rows itself (tile::gather4 by token id, one copy of four
+// rows per lane) instead of reading x pre-gathered into plan order by a separate launch.  It pays with
+// 128-row token tiles (batch: up 2336 -> 2220 us, the gather launch gone) and not with 256-row tiles,
+// where 32 gather copies per stage and CTA hold the producer back (prefill up 2957 -> 3684 us).
+// MOE_PAIR_GATHER=0|1 overrides (the tests cover both).
+bool want_pair_gather(const moe_shape_t& s) {
+  if (const char* env = std::getenv("MOE_PAIR_GATHER")) return std::strcmp(env, "1") == 0;
+  return pair_nmax(s) == 128;
+}
+
+// Whether the up projection of this shape launches the x gather into plan order first.
+bool up_pregathers(const moe_shape_t& s) {
+  if (!want_pregather(s)) return false;
+  const bool pair_path = want_persistent(s) && pair_nmax(s) != 0 && s.I % 256 == 0;
+  return !(pair_path && want_pair_gather(s));
+}
+
 moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan, const moe_shape_t& s,
                     moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t stream) {
   CUtensorMap mg, mu, mx;
@@ -245,6 +262,22 @@ moe_status_t run_up(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_
   const bool gathered = want_pregather(s) && have_ws;
   if (!make_map_bf16(&mg, w->gate, rows, s.H, 128) || !make_map_bf16(&mu, w->up, rows, s.H, 128))
     return MOE_ERR_CUDA;
+  if (persistent && gathered && pair_nmax(s) != 0 && s.I % 256 == 0 && want_pair_gather(s)) {
+    if (!make_map_bf16(&mx, x, s.M, s.H, 1)) return MOE_ERR_CUDA;
+    GroupedGemmArgs a{};
+    a.sorted_ids = plan->sorted_ids;
+    a.expert_counts = plan->expert_counts;
+    a.expert_offsets = plan->expert_offsets;
+    a.out = h;
+    a.err = err;
+    a.M = s.M;
+    a.E = s.E;
+    a.top_k = s.top_k;
+    a.rows_per_expert = s.I;
+    a.kdim = s.H;
+    a.out_ld = s.I;
+    return cuda_status(moe::launch_pair_up(mg, mu, mx, a, pair_nmax(s), num_sms(), stream, true));
+  }
   if (gathered) {
     auto* xg = static_cast<moe_bf16_t*>(ws);
     const cudaError_t e = moe::launch_gather_rows(x, plan->sorted_ids, plan->num_tokens_post_padded, s.M, s.top_k,
@@ -816,7 +849,7 @@ int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype) {
     return 10;
   if (want_fused_layer(s, dtype)) return 1;  // the whole layer in one launch
   if (want_self_route(s, dtype)) return 5;   // router x2, up with the plan, down, finalize
-  return 6 + (want_pregather(s) ? 1 : 0);   // router x2, align, [gather x], up, down, finalize
+  return 6 + (up_pregathers(s) ? 1 : 0);    // router x2, align, [gather x], up, down, finalize
 }
 
 moe_status_t moe_quantize_nvfp4(const moe_bf16_t* src, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* codes,

@@ -42,6 +42,20 @@
 #include "tile_list.cuh"
 
 namespace moe {
+
+#ifdef MOE_PAIR_TRACE
+// Timeline build (MOE_PAIR_TRACE, a separate library made by build.py --trace; never the
+// default): per tile, 8 stamps of the leader CTA -- [0] e | w << 12 | t << 20 | N << 28 | sm << 48,
+// [1] MMA start (accumulator free), [2] first stage ready, [3] last MMA issued, [4] epilogue
+// start, [5] accumulator released, [6] / [7] first / last weight stage issued; [up, down].
+constexpr int kTraceTiles = 8192;
+__device__ unsigned long long g_pair_trace[2][kTraceTiles][8];
+#define MOE_TRACE_STAMP(kind, tile, slot, value) \
+  (g_pair_trace[(kind)][(tile) < kTraceTiles ? (tile) : kTraceTiles - 1][(slot)] = (value))
+#else
+#define MOE_TRACE_STAMP(kind, tile, slot, value) ((void)0)
+#endif
+
 namespace {
 
 constexpr int kBM = 128;                  // weight rows per CTA (MMA M = 256 per pair)
@@ -95,6 +109,17 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_
       : "memory");
 }
 
+// Four rows (arbitrary row indices, one-row boxes) into this CTA's shared memory as four consecutive
+// box rows; the bytes complete on the mbarrier at cluster address `bar` (the leader's).
+__device__ __forceinline__ void tma_gather4_pair(const CUtensorMap* map, uint32_t bar, void* dst, int32_t c0,
+                                                 int32_t r0, int32_t r1, int32_t r2, int32_t r3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot_smem)),
                "r"(ncols)
@@ -134,7 +159,10 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
-template <bool kUp, int kNmax, int kStagesA, int kStagesB>
+// kGatherB (up only): the token rows are gathered from x by token id inside the GEMM (tile::gather4,
+// four rows per copy, one copy per lane) instead of read as consecutive rows of x pre-gathered into
+// plan order.
+template <bool kUp, int kNmax, int kStagesA, int kStagesB, bool kGatherB = false>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_a1,
                      const __grid_constant__ CUtensorMap tm_b, const GroupedGemmArgs args) {
@@ -229,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           alive = false;
           break;
         }
+        if (lane == 0 && leader && (k == 0 || k == nk - 1))
+          MOE_TRACE_STAMP(kUp ? 0 : 1, tile, k == 0 ? 6 : 7, global_timer_ns());
         uint8_t* st = a_ring + s * C::kAStage;
         const uint32_t bar = cluster_addr(&a_full[s], 0);
         if (lane == 0)
@@ -251,12 +281,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int half = N / 2;
       const int row0 = args.expert_offsets[c.e] + c.t * kNmax + static_cast<int>(rank) * half;
       const int nbox = (half + kBRows - 1) / kBRows;
+      // gathered: lane i copies rows 4i .. 4i + 3 of this CTA's half (rows past the expert's count take
+      // token 0; their columns of the product are never stored)
+      int tok[4] = {0, 0, 0, 0};
+      if (kGatherB) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * lane + u;
+          if (r < half && static_cast<int>(rank) * half + r < nrows) {
+            const int id = args.sorted_ids[row0 + r];
+            tok[u] = (id >= 0 && id < nslots) ? id / args.top_k : 0;
+          }
+        }
+      }
+      const uint32_t b_bytes = kGatherB ? 2u * half * kBK * 2 : 2u * nbox * kBRows * kBK * 2;
       for (int k = 0; k < nk; ++k, ++kb) {
         const int s = kb % kStagesB;
         bool ok = true;
         if (lane == 0) {
           ok = mbar_wait_bounded(&b_empty[s], ((kb / kStagesB) & 1) ^ 1, abort_flag);
-          if (ok && leader) mbar_arrive_expect_tx(&b_full[s], 2 * nbox * kBRows * kBK * 2);
+          if (ok && leader) mbar_arrive_expect_tx(&b_full[s], b_bytes);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
@@ -268,9 +312,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* st = b_ring + s * C::kBStage;
-        if (lane < nbox)
+        if (kGatherB) {
+          if (4 * lane < half)
+            tma_gather4_pair(&tm_b, cluster_addr(&b_full[s], 0), st + lane * 4 * kBK * 2, k * kBK, tok[0], tok[1],
+                             tok[2], tok[3], pol_b);
+        } else if (lane < nbox) {
           tma_load_2d_pair(&tm_b, cluster_addr(&b_full[s], 0), st + lane * kBRows * kBK * 2, k * kBK,
                            row0 + lane * kBRows, pol_b);
+        }
       }
     }
     __syncwarp();
@@ -284,6 +333,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nrows = min(kNmax, cnt[c.e] - c.t * kNmax);
         const int N = (nrows + 15) & ~15;
         const uint32_t idesc = umma_idesc_bf16(2 * kBM, N);
+#ifdef MOE_PAIR_TRACE
+        {
+          unsigned smid;
+          asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+          MOE_TRACE_STAMP(kUp ? 0 : 1, tile, 0,
+                          static_cast<unsigned long long>(c.e) | (static_cast<unsigned long long>(c.w) << 12) |
+                              (static_cast<unsigned long long>(c.t) << 20) |
+                              (static_cast<unsigned long long>(N) << 28) |
+                              (static_cast<unsigned long long>(smid) << 48));
+        }
+#endif
         const int buf = j % C::kAccBufs;
         const int use = j / C::kAccBufs;
         if (!mbar_wait_bounded(&acc_empty[buf], (use & 1) ^ 1, abort_flag)) {
@@ -292,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after_sync();
+        MOE_TRACE_STAMP(kUp ? 0 : 1, tile, 1, global_timer_ns());
         const uint32_t d0 = tmem + buf * C::kAccCols;
         const uint32_t d1 = d0 + kNmax;
         for (int k = 0; k < nk; ++k, ++ka, ++kb) {
@@ -304,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after_sync();
+          if (k == 0) MOE_TRACE_STAMP(kUp ? 0 : 1, tile, 2, global_timer_ns());
           const uint64_t da0 = umma_desc_sw128(a_ring + sa * C::kAStage);
           const uint64_t da1 = umma_desc_sw128(a_ring + sa * C::kAStage + kBoxBytes);
           const uint64_t db = umma_desc_sw128(b_ring + sb * C::kBStage);
@@ -316,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit_pair(&a_empty[sa]);
           umma_commit_pair(&b_empty[sb]);
         }
+        MOE_TRACE_STAMP(kUp ? 0 : 1, tile, 3, global_timer_ns());
         umma_commit_pair(&acc_full[buf]);  // also on an abort, so neither epilogue is left waiting
       }
     }
@@ -333,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = j % C::kAccBufs;
       bool ok = true;
       if (lane == 0) ok = mbar_wait_bounded(&acc_full[buf], (j / C::kAccBufs) & 1, abort_flag);
+      if (lane == 0 && warp == 4 && leader) MOE_TRACE_STAMP(kUp ? 0 : 1, tile, 4, global_timer_ns());
       ok = __shfl_sync(0xffffffffu, ok, 0);
       tc_fence_after_sync();
       const bool go = __shfl_sync(0xffffffffu, ok && !*abort_flag, 0);
@@ -341,63 +405,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
-      int ids[kNmax / 32];
-      if (!kUp) {
-#pragma unroll
-        for (int i = 0; i < kNmax / 32; ++i) {
-          const int n = lane + 32 * i;
-          ids[i] = (n < nrows) ? args.sorted_ids[row0 + n] : -1;
-        }
-      }
       const int colbase = kUp ? c.w * 2 * kBM + static_cast<int>(rank) * kBM
                               : c.w * 4 * kBM + static_cast<int>(rank) * kBM;
-      // lane l holds column col0 + l (its tensor-memory lane) for the tokens of each 16-column chunk;
-      // 8 x 8 transposes inside each group of 8 lanes give lane (8 g + b) token b's columns
-      // col0 + 8 g .. + 7, written as one 16-byte store per 8 tokens
-      const int g8 = lane >> 3, b8 = lane & 7;
-      const int col8 = colbase + q * 32 + 8 * g8;
-      for (int cb = 16 * part_c; cb < N; cb += 64) {
+      // 1. drain: lane l holds column col0 + l (its tensor-memory lane) for the tokens of each of the
+      //    warp's 16-column chunks; the results are packed as bf16 token pairs in registers and the
+      //    accumulator is released at once, so the next tile's MMAs run while this tile is stored
+      constexpr int kChunks = kNmax / 64;
+      constexpr int kWords = kUp ? 8 : 16;  // bf16 token pairs per chunk (down: both 256-row halves)
+      uint32_t pk[kChunks][kWords];
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int cb = 16 * part_c + 64 * i;
+        if (cb >= N) break;
         uint32_t v0[16], v1[16];
         tmem_load_16(lane_base + cb, v0);
         tmem_load_16(lane_base + kNmax + cb, v1);
         tmem_load_wait();
-        const int id_word = kUp ? 0 : pick<kNmax / 32>(ids, cb >> 5);
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const int n = cb + 8 * m + b8;  // the token this lane writes after the transpose
+        for (int p = 0; p < 8; ++p) {
           if (kUp) {
-            uint32_t hv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float g = __uint_as_float(v0[8 * m + i]);
-              const float u = __uint_as_float(v1[8 * m + i]);
-              hv[i] = bf16_bits_rn(silu_mul(g, u));
-            }
-            transpose8x8(hv, b8);
-            if (n < nrows)
-              *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(row0 + n) * args.out_ld + col8) =
-                  pack8_bf16(hv);
+            pk[i][p] = pack_bf16x2(silu_mul(__uint_as_float(v0[2 * p]), __uint_as_float(v1[2 * p])),
+                                   silu_mul(__uint_as_float(v0[2 * p + 1]), __uint_as_float(v1[2 * p + 1])));
           } else {
-            uint32_t a[8], bb[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              a[i] = bf16_bits_rn(__uint_as_float(v0[8 * m + i]));
-              bb[i] = bf16_bits_rn(__uint_as_float(v1[8 * m + i]));
-            }
-            transpose8x8(a, b8);
-            transpose8x8(bb, b8);
-            const int id = __shfl_sync(0xffffffffu, id_word, (cb & 31) + 8 * m + b8);
-            if (n < nrows && id >= 0 && id < nslots) {
-              uint16_t* yr = args.out + static_cast<size_t>(id) * args.out_ld + col8;
-              *reinterpret_cast<uint4*>(yr) = pack8_bf16(a);
-              *reinterpret_cast<uint4*>(yr + 2 * kBM) = pack8_bf16(bb);
-            }
+            pk[i][p] = pack_bf16x2(__uint_as_float(v0[2 * p]), __uint_as_float(v0[2 * p + 1]));
+            pk[i][8 + p] = pack_bf16x2(__uint_as_float(v1[2 * p]), __uint_as_float(v1[2 * p + 1]));
           }
         }
       }
       tc_fence_before_sync();
       __syncwarp();
+      if (lane == 0 && warp == 4 && leader) MOE_TRACE_STAMP(kUp ? 0 : 1, tile, 5, global_timer_ns());
       if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[buf], 0));
+      // 2. store: an 8 x 8 transpose of the packed words inside each group of 8 lanes gives lane
+      //    (8 g + b) tokens 2b and 2b + 1 of the chunk at columns col0 + 8 g .. + 7: two 16-byte
+      //    row stores per lane per 16 tokens
+      const int g8 = lane >> 3, b8 = lane & 7;
+      const int col8 = colbase + q * 32 + 8 * g8;
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int cb = 16 * part_c + 64 * i;
+        if (cb >= N) break;
+        const int n0 = cb + 2 * b8, n1 = n0 + 1;
+        int id0 = -1, id1 = -1;  // down: the slots these two tokens' rows go to
+        if (!kUp) {
+          if (n0 < nrows) id0 = args.sorted_ids[row0 + n0];
+          if (n1 < nrows) id1 = args.sorted_ids[row0 + n1];
+        }
+#pragma unroll
+        for (int half = 0; half < (kUp ? 1 : 2); ++half) {
+          uint32_t w[8];
+#pragma unroll
+          for (int p = 0; p < 8; ++p) w[p] = pk[i][8 * half + p];
+          transpose8x8(w, b8);
+          const uint4 r0 = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                      __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+          const uint4 r1 = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                      __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+          if (kUp) {
+            if (n0 < nrows)
+              *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(row0 + n0) * args.out_ld + col8) = r0;
+            if (n1 < nrows)
+              *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(row0 + n1) * args.out_ld + col8) = r1;
+          } else {
+            const int cc = col8 + half * 2 * kBM;
+            if (n0 < nrows && id0 >= 0 && id0 < nslots)
+              *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(id0) * args.out_ld + cc) = r0;
+            if (n1 < nrows && id1 >= 0 && id1 < nslots)
+              *reinterpret_cast<uint4*>(args.out + static_cast<size_t>(id1) * args.out_ld + cc) = r1;
+          }
+        }
+      }
     }
   }
   tc_fence_before_sync();
@@ -406,11 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
-template <bool kUp, int kNmax, int kStagesA, int kStagesB>
+template <bool kUp, int kNmax, int kStagesA, int kStagesB, bool kGatherB = false>
 cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const GroupedGemmArgs& args,
                         int num_sms, cudaStream_t stream) {
   using C = QCfg<kNmax, kStagesA, kStagesB>;
-  auto kern = pair_gemm_kernel<kUp, kNmax, kStagesA, kStagesB>;
+  auto kern = pair_gemm_kernel<kUp, kNmax, kStagesA, kStagesB, kGatherB>;
   int dev = 0;
   cudaError_t st = cudaGetDevice(&dev);
   if (st != cudaSuccess) return st;
@@ -438,8 +515,12 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
 }  // namespace
 
 cudaError_t launch_pair_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
-                           const GroupedGemmArgs& args, int nmax, int num_sms, cudaStream_t stream) {
+                           const GroupedGemmArgs& args, int nmax, int num_sms, cudaStream_t stream, bool gather_b) {
   if (args.rows_per_expert % (2 * kBM) != 0) return cudaErrorInvalidValue;
+  if (gather_b) {
+    if (nmax >= 256) return launch_pair<true, 256, 5, 3, true>(w_gate, w_up, x_rows, args, num_sms, stream);
+    return launch_pair<true, 128, 5, 6, true>(w_gate, w_up, x_rows, args, num_sms, stream);
+  }
   if (nmax >= 256) return launch_pair<true, 256, 5, 3>(w_gate, w_up, x_rows, args, num_sms, stream);
   return launch_pair<true, 128, 5, 6>(w_gate, w_up, x_rows, args, num_sms, stream);
 }
@@ -452,3 +533,15 @@ cudaError_t launch_pair_down(const CUtensorMap& w_down, const CUtensorMap& h_row
 }
 
 }  // namespace moe
+
+#ifdef MOE_PAIR_TRACE
+// Host access to the timeline of the last pair launches (trace build only).
+extern "C" __attribute__((visibility("default"))) int moe_pair_trace_read(void* host, size_t bytes) {
+  return cudaMemcpyFromSymbol(host, moe::g_pair_trace, bytes) == cudaSuccess ? 0 : 1;
+}
+extern "C" __attribute__((visibility("default"))) int moe_pair_trace_clear() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, moe::g_pair_trace) != cudaSuccess) return 1;
+  return cudaMemset(p, 0, sizeof(moe::g_pair_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif

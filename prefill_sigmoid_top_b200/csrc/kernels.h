@@ -87,7 +87,8 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* sorted_ids, con
 // `nmax` plan rows (128 or 256) split over the two CTAs of a cluster; the
 // token-row tensor is plan-ordered (x gathered, or h) in 32-row boxes.
 cudaError_t launch_pair_up(const CUtensorMap& w_gate, const CUtensorMap& w_up, const CUtensorMap& x_rows,
-                           const GroupedGemmArgs& args, int nmax, int num_sms, cudaStream_t stream);
+                           const GroupedGemmArgs& args, int nmax, int num_sms, cudaStream_t stream,
+                           bool gather_b = false);
 cudaError_t launch_pair_down(const CUtensorMap& w_down, const CUtensorMap& h_rows, const GroupedGemmArgs& args,
                              int nmax, int num_sms, cudaStream_t stream);
 

@@ -209,7 +209,11 @@ __device__ void locate_tile(const int* s_cnt, int E, int ti, int* s_info) {
 // NVFP4 copy of h (plan order, `cols` wide): codes and scale atoms.  Rows past
 // the expert's count are not written: the GEMM computes their columns from
 // whatever they hold and never stores them (a column of the product depends
-// on its own row of this operand only).
+// on its own row of this operand only).  Each thread takes 64 consecutive
+// elements of one row (four 16-element blocks): eight 16-byte loads, two
+// 16-byte code stores, and the four scales as one 32-bit word (four column
+// blocks of one atom row are adjacent bytes); blockIdx.y splits the row's
+// 64-element groups over a few CTAs per tile.
 __global__ void __launch_bounds__(256) quantize_tiles_kernel(
     const uint16_t* __restrict__ src, const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int E,
     int cols, const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ atoms) {
@@ -226,21 +230,28 @@ __global__ void __launch_bounds__(256) quantize_tiles_kernel(
   const int nrows = min(128, s_cnt[e] - local * 128);
   const int row0 = offsets[e] + local * 128;
   const float gs = nvfp4_global_scale(__uint_as_float(*amax_bits));
-  const int nblk = cols / 16;
-  // this CTA's slice of 16-element column blocks: [jb0, jb1)
-  const int per = (nblk + gridDim.y - 1) / gridDim.y;
-  const int jb0 = blockIdx.y * per, jb1 = min(nblk, jb0 + per);
-  const int width = jb1 - jb0;
+  const int ngrp = cols / 64;  // 64-element groups per row
+  // this CTA's slice of the groups: [g0, g1)
+  const int per = (ngrp + gridDim.y - 1) / gridDim.y;
+  const int g0 = blockIdx.y * per, g1 = min(ngrp, g0 + per);
+  const int width = g1 - g0;
   for (int idx = tid; idx < nrows * width; idx += blockDim.x) {
     const int r = idx / width;
-    const int j = jb0 + (idx - r * width);
-    float v[16];
-    load16_bf16(src + static_cast<int64_t>(row0 + r) * cols + j * 16, v);
-    uint32_t packed[2];
-    const uint8_t sc = quantize_block16(v, gs, packed);
-    *reinterpret_cast<uint2*>(codes + (static_cast<int64_t>(ti) * 128 + r) * (cols / 2) + j * 8) =
-        make_uint2(packed[0], packed[1]);
-    atoms[(static_cast<int64_t>(ti) * (cols / 64) + j / 4) * 512 + (r % 32) * 16 + (r / 32) * 4 + (j % 4)] = sc;
+    const int gi = g0 + (idx - r * width);
+    const uint16_t* row = src + static_cast<int64_t>(row0 + r) * cols + gi * 64;
+    uint32_t packed[4][2];
+    uint32_t scw = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float v[16];
+      load16_bf16(row + b * 16, v);
+      scw |= static_cast<uint32_t>(quantize_block16(v, gs, packed[b])) << (8 * b);
+    }
+    uint8_t* cdst = codes + (static_cast<int64_t>(ti) * 128 + r) * (cols / 2) + gi * 32;
+    reinterpret_cast<uint4*>(cdst)[0] = make_uint4(packed[0][0], packed[0][1], packed[1][0], packed[1][1]);
+    reinterpret_cast<uint4*>(cdst)[1] = make_uint4(packed[2][0], packed[2][1], packed[3][0], packed[3][1]);
+    *reinterpret_cast<uint32_t*>(atoms + (static_cast<int64_t>(ti) * ngrp + gi) * 512 + (r % 32) * 16 +
+                                 (r / 32) * 4) = scw;
   }
 }
 
@@ -580,41 +591,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_one(acc_empty);  // tensor memory is free for the next tile
       const float s0 = args.gs_a0[c.e] * act_gs;
       const float s1 = args.gs_a1[c.e] * act_gs;
-      int ids[4];
-      if (!kUp) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int n = lane + 32 * i;
-          ids[i] = (n < nrows) ? g.sorted_ids[row0 + n] : -1;
-        }
-      }
-      auto* out = reinterpret_cast<__nv_bfloat16*>(g.out);
+      // lane l holds column col0 + l for the 16 tokens of each chunk: pack token pairs as bf16,
+      // transpose 8 x 8 inside each group of 8 lanes, and lane (8 g + b) writes tokens 2b and 2b + 1
+      // at columns col0 + 8 g .. + 7 with one 16-byte store each
+      const int g8 = lane >> 3, b8 = lane & 7;
+      const int col8 = (kUp ? c.w * kBM : c.w * 2 * kBM) + q * 32 + 8 * g8;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int cb = 16 * (2 * i + half);
         if (cb >= N) break;
-        const int w4 = cb >> 5;  // which 32-row group of slot ids
-        const int id_word = kUp ? 0 : (w4 == 0 ? ids[0] : w4 == 1 ? ids[1] : w4 == 2 ? ids[2] : ids[3]);
+        const int n0 = cb + 2 * b8, n1 = n0 + 1;
+        int id0 = -1, id1 = -1;
+        if (!kUp) {
+          if (n0 < nrows) id0 = g.sorted_ids[row0 + n0];
+          if (n1 < nrows) id1 = g.sorted_ids[row0 + n1];
+        }
 #pragma unroll
-        for (int qq = 0; qq < 16; ++qq) {
-          const int n = cb + qq;
+        for (int part = 0; part < (kUp ? 1 : 2); ++part) {
+          uint32_t w[8];
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            if (kUp) {
+              float hv[2];
+#pragma unroll
+              for (int u2 = 0; u2 < 2; ++u2) {
+                const int qq = 2 * p + u2;
+                const float gt = __uint_as_float(v0[i][qq]) * s0;
+                const float ut = __uint_as_float(v1[i][qq]) * s1;
+                hv[u2] = silu_mul(gt, ut);
+              }
+              w[p] = pack_bf16x2(hv[0], hv[1]);
+              if (cb + 2 * p < nrows) hmax = fmaxf(hmax, fabsf(bf16_lo(w[p])));
+              if (cb + 2 * p + 1 < nrows) hmax = fmaxf(hmax, fabsf(bf16_hi(w[p])));
+            } else {
+              const uint32_t* v = part == 0 ? v0[i] : v1[i];
+              const float sc = part == 0 ? s0 : s1;
+              w[p] = pack_bf16x2(__uint_as_float(v[2 * p]) * sc, __uint_as_float(v[2 * p + 1]) * sc);
+            }
+          }
+          transpose8x8(w, b8);
+          const uint4 r0 = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                      __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+          const uint4 r1 = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                      __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
           if (kUp) {
-            if (n < nrows) {
-              const float gt = __uint_as_float(v0[i][qq]) * s0;
-              const float ut = __uint_as_float(v1[i][qq]) * s1;
-              const int col = c.w * kBM + q * 32 + lane;
-              const __nv_bfloat16 hv = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * ut);
-              out[static_cast<size_t>(row0 + n) * g.out_ld + col] = hv;
-              hmax = fmaxf(hmax, fabsf(__bfloat162float(hv)));
-            }
+            if (n0 < nrows) *reinterpret_cast<uint4*>(g.out + static_cast<size_t>(row0 + n0) * g.out_ld + col8) = r0;
+            if (n1 < nrows) *reinterpret_cast<uint4*>(g.out + static_cast<size_t>(row0 + n1) * g.out_ld + col8) = r1;
           } else {
-            const int id = __shfl_sync(0xffffffffu, id_word, (cb & 31) + qq);
-            if (n < nrows && id >= 0 && id < nslots) {
-              const int col = c.w * 2 * kBM + q * 32 + lane;
-              out[static_cast<size_t>(id) * g.out_ld + col] = __float2bfloat16_rn(__uint_as_float(v0[i][qq]) * s0);
-              out[static_cast<size_t>(id) * g.out_ld + col + kBM] =
-                  __float2bfloat16_rn(__uint_as_float(v1[i][qq]) * s1);
-            }
+            const int cc = col8 + part * kBM;
+            if (n0 < nrows && id0 >= 0 && id0 < nslots)
+              *reinterpret_cast<uint4*>(g.out + static_cast<size_t>(id0) * g.out_ld + cc) = r0;
+            if (n1 < nrows && id1 >= 0 && id1 < nslots)
+              *reinterpret_cast<uint4*>(g.out + static_cast<size_t>(id1) * g.out_ld + cc) = r1;
           }
         }
       }
@@ -692,7 +720,7 @@ cudaError_t launch_amax_plan_rows(const uint16_t* h, const int32_t* sorted_ids, 
 cudaError_t launch_quantize_tiles(const uint16_t* src, const int32_t* counts, const int32_t* offsets, int E, int cols,
                                   int tiles_ub, const unsigned* amax_bits, uint8_t* codes, uint8_t* atoms,
                                   cudaStream_t stream) {
-  const int slices = std::max(1, cols / 16 / 16);  // 16 column blocks (256 elements) per CTA
+  const int slices = std::max(1, cols / 512);  // 8 groups of 64 elements per CTA and row
   quantize_tiles_kernel<<<dim3(tiles_ub, slices), 256, 0, stream>>>(src, counts, offsets, E, cols, amax_bits, codes,
                                                                     atoms);
   return cudaGetLastError();

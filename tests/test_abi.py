@@ -172,6 +172,11 @@ def test_layer_kernel_count(monkeypatch):
     many_experts = moe.Shape(M=2, H=7168, I=2048, E=512, top_k=8, block_size=16)
     assert moe.layer_kernel_count(many_experts) == 5  # the single launch takes E <= 256
     batch = moe.Shape(M=512, H=7168, I=2048, E=256, top_k=16, block_size=64)
-    assert moe.layer_kernel_count(batch) == 7         # align and a gather pass of x
+    assert moe.layer_kernel_count(batch) == 6         # align; the up kernel gathers x rows itself
+    prefill = moe.Shape(M=2048, H=7168, I=2048, E=256, top_k=16, block_size=128)
+    assert moe.layer_kernel_count(prefill) == 7       # align and a gather pass of x (256-row token tiles)
+    monkeypatch.setenv("MOE_PAIR_GATHER", "0")
+    assert moe.layer_kernel_count(batch) == 7
+    monkeypatch.delenv("MOE_PAIR_GATHER")
     assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 10
     assert moe.layer_kernel_count(moe.Shape(M=16, H=255, I=128, E=8, top_k=2, block_size=16)) == -1

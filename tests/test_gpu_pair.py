@@ -3,7 +3,8 @@
 Same bars as the single-SM grouped projections: h and y elementwise within 2^-7 |ref| + 1e-2 RMS(ref)
 against the oracle's bf16-rounded values, padding rows of h never written, canaries intact, no device
 error.  The cases cover token tiles narrower than a box (8 rows per CTA), several 256-row tiles per
-expert with a ragged tail, empty experts, and both token-tile widths.
+expert with a ragged tail, empty experts, both token-tile widths, and x rows either pre-gathered into
+plan order or gathered by the up kernel itself (tile::gather4).
 """
 import numpy as np
 import pytest
@@ -25,9 +26,11 @@ PAIR_CASES = [
 ]
 
 
+@pytest.mark.parametrize("gather", ["0", "1"])
 @pytest.mark.parametrize("pair", ["128", "256"])
 @pytest.mark.parametrize("case", PAIR_CASES)
-def test_pair_up_down(case, pair, monkeypatch):
+def test_pair_up_down(case, pair, gather, monkeypatch):
+    monkeypatch.setenv("MOE_PAIR_GATHER", gather)  # x rows pre-gathered into plan order, or gathered in the GEMM
     monkeypatch.setenv("MOE_GEMM_PERSISTENT", "1")
     monkeypatch.setenv("MOE_UP_GATHER", "pregather")
     monkeypatch.setenv("MOE_GEMM_NMAX", "128")

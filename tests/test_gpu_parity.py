@@ -70,8 +70,11 @@ SMALL_ROUTER_SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("tile", ["default", "0"])  # many-token CTA tile: 4 x 2 warps (default) or 2 x 2
 @pytest.mark.parametrize("M,H,E,K,bias", SMALL_ROUTER_SHAPES)
-def test_router_bitexact_small(M, H, E, K, bias):
+def test_router_bitexact_small(M, H, E, K, bias, tile, monkeypatch):
+    if tile != "default":
+        monkeypatch.setenv("MOE_ROUTER_TILE", tile)
     cfg = inputs.WORKLOADS[0].with_(M=M, H=H, E=E, K=K, bias=bias, seed=M * 7 + E)
     w_r, b, g, x = inputs.router_inputs(cfg)
     ids, w = moe.route(x.to(DEV), w_r.to(DEV), b.to(DEV), K)
