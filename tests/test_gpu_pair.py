@@ -23,6 +23,8 @@ PAIR_CASES = [
     dict(M=600, H=512, I=512, E=4, K=2, B=16),     # 300 rows per expert: 256-row tiles plus a ragged tail
     dict(M=40, H=1024, I=256, E=16, K=4, B=16),    # ~10 rows per expert: 8 rows per CTA
     dict(M=5, H=512, I=256, E=64, K=6, B=32),      # most experts empty
+    dict(M=600, H=1024, I=512, E=4, K=2, B=16),    # two weight blocks per expert in both projections
+    dict(M=64, H=1024, I=1024, E=8, K=4, B=16),    # ~32 rows per expert over four up weight blocks
 ]
 
 
