@@ -48,11 +48,21 @@ NCU_TRAFFIC = {
     # decode M=8, the single-launch layer: E=32 capture (2.7368 GB read + write for 31 touched
     # experts, 1.0020 x its 2.7312 GB of algorithmic bytes) scaled to 95 touched experts
     (1, "layer_fused"): (8_386_900_000, "d815c00a1de4a117"),
+    # batch M=512 and prefill M=2048: the up projection (2-SM pair kernel) captured at full size, one pass
+    # (dram__bytes_read.sum + dram__bytes_write.sum of one launch)
+    (2, "pair_up"): (15_305_074_944, "5c0cd642d8591f67"),
+    (3, "pair_up"): (16_934_910_208, "5c0cd642d8591f67"),
+    # NVFP4 M=1000: the block-scaled up projection captured at full size, one pass
+    (4, "nvfp4_up"): (4_656_227_584, "cc73a5d8c3d56c67"),
 }
 KERNEL_SOURCES = {
     "up": ["prefill_sigmoid_top_b200/csrc/gemm_bf16.cu", "prefill_sigmoid_top_b200/csrc/common.cuh"],
     "layer_fused": ["prefill_sigmoid_top_b200/csrc/layer_fused.cu", "prefill_sigmoid_top_b200/csrc/common.cuh",
                     "prefill_sigmoid_top_b200/csrc/router_dot.cuh"],
+    "pair_up": ["prefill_sigmoid_top_b200/csrc/gemm_pair.cu", "prefill_sigmoid_top_b200/csrc/common.cuh",
+                "prefill_sigmoid_top_b200/csrc/tile_list.cuh"],
+    "nvfp4_up": ["prefill_sigmoid_top_b200/csrc/nvfp4.cu", "prefill_sigmoid_top_b200/csrc/common.cuh",
+                 "prefill_sigmoid_top_b200/csrc/tile_list.cuh"],
 }
 
 
@@ -86,6 +96,9 @@ def parse_args(argv=None):
     p.add_argument("--route-only", action="store_true",
                    help="time moe_route alone on the workload's router inputs (no expert weights allocated; "
                         "a small target for profiler captures of the router kernels)")
+    p.add_argument("--probe-tma", action="store_true",
+                   help="time the TMA weight-panel stream of the grouped GEMMs without their MMAs "
+                        "(moe_measure_tma_stream) from HBM and from L2, beside the plain streaming read")
     return p.parse_args(argv)
 
 
@@ -529,8 +542,11 @@ def measure_workload(cfg, args, dev, world, rank, want_cpu, read_ceiling_box):
                "achieved": ab["layer"] / (ms_per_step / 1e3) / 1e9, "algorithmic_bytes": ab["layer"],
                "traffic": ncu_traffic("layer_fused")}
     else:
-        dom = {"kernel": "grouped_up_swiglu (staged pass)", "achieved": up_achieved,
-               "algorithmic_bytes": ab["up"], "traffic": None}
+        pair = (not nvfp4) and cid in (2, 3)
+        name = ": pair_gemm_kernel<up>" if pair else (": persistent_nvfp4_kernel<up>" if nvfp4 else "")
+        dom = {"kernel": "grouped_up_swiglu (staged pass)" + name,
+               "achieved": up_achieved, "algorithmic_bytes": ab["up"],
+               "traffic": ncu_traffic("pair_up") if pair else (ncu_traffic("nvfp4_up") if nvfp4 else None)}
     dom.update(bound="hbm", peak=hbm_peak, unit="GB/s", frac=dom["achieved"] / hbm_peak, peak_source=peak_kind)
     if read_ceiling_box.get("gbs"):
         dom["read_ceiling_gbs"] = read_ceiling_box["gbs"]
@@ -792,6 +808,56 @@ def run_tp_emulated(args):
                       "steps": args.steps}), flush=True)
 
 
+# (boxes per stage, stages in flight, contiguous, issuing warps): one 16 KB box per stage as a single panel
+# walk; two boxes per stage as the up kernels' gate + up panels (the 2-SM pair kernels: 5 stages, one
+# issuing thread); three boxes; and the two-box walk taken in turn by 2 and 4 issuing warps
+TMA_PROBES = [(1, 10, False, 1), (2, 5, False, 1), (3, 4, False, 1), (1, 10, True, 1), (2, 5, True, 1),
+              (3, 4, True, 1), (2, 6, False, 2), (2, 4, False, 4), (3, 4, False, 4)]
+
+
+def run_probe_tma(args):
+    """The weight-panel stream of the grouped GEMMs on its own: one CTA per SM copying 128 x 64 bf16 boxes
+    of 128-row panels into a ring of shared-memory stages (moe_measure_tma_stream), from an 8 GB buffer
+    (HBM) and from its first 32 MB (resident in L2), for the probes of TMA_PROBES; best of 3 device-timed
+    calls each, beside the plain streaming read of the same 8 GB.  A measurement of the memory system, not
+    of the layer."""
+    import torch
+    import prefill_sigmoid_top_b200 as moe
+    buf = torch.ones(8 << 30, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rows = []
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            moved = fn()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1) * 1e-3)
+        return moved, best
+
+    for where, view in (("hbm", buf), ("l2", buf[: 32 << 20])):
+        for boxes, stages, contiguous, warps in TMA_PROBES:
+            steps = max(stages, int((4 << 30) / (148 * boxes * 16384)))
+            moved, sec = timed(lambda: moe.measure_tma_stream(view, boxes, stages, contiguous, steps, err,
+                                                              warps=warps))
+            rows.append({"source": where, "boxes_per_stage": boxes, "stages": stages, "issuing_warps": warps,
+                         "copy": "bulk 16 KB (panel stored box by box)" if contiguous else "2-D tensor box 128 x 64",
+                         "in_flight_kb_per_sm": boxes * stages * 16, "GBps": moved / sec / 1e9,
+                         "us_per_stage": sec * 1e6 / steps})
+    if moe.get_device_error(err) != 0:
+        raise RuntimeError("moe_measure_tma_stream: a bounded wait expired")
+    read_gbs = measure_read_ceiling(moe, torch, buf)
+    print(json.dumps({"kernel": "tma_stream_kernel (moe_measure_tma_stream)",
+                      "ctas": "one per SM; one thread per issuing warp waits and issues",
+                      "panel": "128 rows x 7168 bf16 columns, 64-column steps", "hbm_read_ceiling_gbs": read_gbs,
+                      "probes": rows}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -800,6 +866,8 @@ def main(argv=None):
         run_tp_emulated(args)
     elif args.route_only:
         run_route_only(args)
+    elif args.probe_tma:
+        run_probe_tma(args)
     else:
         run_ours(args)
 

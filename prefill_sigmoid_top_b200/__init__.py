@@ -115,6 +115,8 @@ def _declare(L):
         "moe_route_noalloc": (st, [vp, vp, vp, _Shape, vp, vp, vp]),
         "moe_selftest_wait_timeout": (st, [vp, ctypes.c_uint32, vp]),
         "moe_measure_hbm_read": (st, [vp, sz, vp, vp]),
+        "moe_measure_tma_stream": (st, [vp, sz, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, vp, ctypes.POINTER(ctypes.c_size_t), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -463,6 +465,21 @@ def measure_hbm_read(buf, sink):
     _need_cuda(buf, sink)
     _check(library().moe_measure_hbm_read(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), _stream()),
            "moe_measure_hbm_read")
+
+
+def measure_tma_stream(buf, boxes: int, stages: int, contiguous: bool, steps: int, err_flag=None,
+                       warps: int = 1) -> int:
+    """Enqueue one TMA weight-panel stream over the tensor ``buf`` (moe_measure_tma_stream: ``boxes``
+    16 KB boxes per stage, ``stages`` stages in flight, 2-D tensor boxes or ``contiguous`` bulk copies,
+    ``warps`` issuing threads per CTA, ``steps`` stages per CTA); returns the bytes the call copies into
+    shared memory."""
+    _need_cuda(buf)
+    moved = ctypes.c_size_t(0)
+    _check(library().moe_measure_tma_stream(_ptr(buf), buf.numel() * buf.element_size(), int(boxes), int(stages),
+                                            1 if contiguous else 0, int(warps), int(steps),
+                                            _ptr(err_flag) if err_flag is not None else None,
+                                            ctypes.byref(moved), _stream()), "moe_measure_tma_stream")
+    return int(moved.value)
 
 
 def get_device_error(err_flag) -> int:

@@ -613,6 +613,10 @@ moe_status_t run_layer_to_y(const moe_bf16_t* x, const moe_bf16_t* w_router, con
 }  // namespace
 
 namespace moe {
+bool encode_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_map_bf16(map, base, rows, cols, box_rows);
+}
+
 int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,
                      const void* topk_w) {
   const moe_status_t st = check_shape(s);

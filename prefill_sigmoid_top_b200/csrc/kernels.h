@@ -11,6 +11,9 @@
 namespace moe {
 
 // api.cu: validation of moe_route's arguments (a moe_status_t value).
+// 2-D bf16 tensor map [rows, cols] with boxes of box_rows x 64 elements and the 128-byte swizzle.
+bool encode_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
 int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,
                      const void* topk_w);
 

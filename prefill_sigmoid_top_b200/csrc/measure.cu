@@ -1,7 +1,9 @@
-// Measurement aid (declared in include/moe_b200_measure.h): a plain streaming
-// read of device memory, the ceiling a read-only weight stream is held to.
+// Measurement aids (declared in include/moe_b200_measure.h): a plain streaming
+// read of device memory, the ceiling a read-only weight stream is held to, and
+// the TMA weight-panel stream of the grouped GEMMs without their MMAs.
 #include "moe_b200_measure.h"
 #include "common.cuh"
+#include "kernels.h"
 
 namespace {
 
@@ -48,4 +50,100 @@ extern "C" moe_status_t moe_measure_hbm_read(const void* buf, size_t bytes, uint
   hbm_read_kernel<<<sms * kCtasPerSm, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(buf), bytes / 16, sink);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// The weight-panel stream of the grouped GEMMs without the GEMM (moe_measure_tma_stream).
+namespace {
+
+constexpr int kPanelRows = 128;
+constexpr int kPanelCols = 7168;                     // bf16 columns of the panel view
+constexpr uint32_t kBox = kPanelRows * 64 * 2;       // one 128 x 64 bf16 box: 16 KB
+constexpr int kMaxStages = 16;
+constexpr uint32_t kMaxRing = 192 * 1024;
+
+struct TmaStreamArgs {
+  const uint8_t* base;
+  long long npanels;
+  int boxes, stages, contiguous, warps, steps;
+  int32_t* err;
+};
+
+// Issuer w (lane 0 of warp w) takes the steps i with i % warps == w.  Step i uses slot i % stages; since
+// stages is a multiple of warps, step i + stages (the next use of that slot) belongs to the same issuer,
+// which issues it only after it has seen step i land, so a slot is never re-armed while its copy is in
+// flight and no issuer waits on a phase another issuer has yet to arm.
+__global__ void __launch_bounds__(128, 1) tma_stream_kernel(const __grid_constant__ CUtensorMap map, TmaStreamArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kMaxStages];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) moe::mbar_init(&full[s], 1);
+    moe::fence_mbar_init();
+  }
+  __syncthreads();
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) != 0 || w >= a.warps) return;  // one thread per issuing warp, as the GEMMs' producers
+  constexpr int nk = kPanelCols / 64;
+  const uint32_t stage_bytes = kBox * static_cast<uint32_t>(a.boxes);
+  // first row of box b's panel at step i: this CTA's sequence of panels, box b offset by half the panels
+  auto panel_row = [&](int i, int b) -> int {
+    const long long pi = static_cast<long long>(blockIdx.x) + static_cast<long long>(i / nk) * gridDim.x;
+    return static_cast<int>(((pi * 7919 + b * (a.npanels / 2)) % a.npanels) * kPanelRows);
+  };
+  auto issue = [&](int i) {
+    const int s = i % a.stages, k = i % nk;
+    moe::mbar_arrive_expect_tx(&full[s], stage_bytes);
+    for (int b = 0; b < a.boxes; ++b) {
+      uint8_t* dst = ring + static_cast<size_t>(s) * stage_bytes + b * kBox;
+      const int row = panel_row(i, b);
+      if (a.contiguous)  // the panel stored box by box: box k is bytes [k * 16 KB, (k + 1) * 16 KB) of the panel
+        moe::bulk_load(dst, a.base + static_cast<size_t>(row) * (kPanelCols * 2) + static_cast<size_t>(k) * kBox, kBox,
+                       &full[s]);
+      else
+        moe::tma_load_2d(&map, &full[s], dst, k * 64, row);
+    }
+  };
+  for (int i = w; i < a.stages && i < a.steps; i += a.warps) issue(i);
+  for (int i = w; i < a.steps; i += a.warps) {
+    const int s = i % a.stages;
+    if (!moe::mbar_wait_bounded(&full[s], (i / a.stages) & 1, nullptr)) {
+      moe::set_error(a.err, moe::kErrTimeout);
+      // this issuer's copies still in flight land before it leaves
+      for (int j = i + a.warps; j < i + a.stages && j < a.steps; j += a.warps)
+        moe::mbar_wait_bounded(&full[j % a.stages], (j / a.stages) & 1, nullptr);
+      return;
+    }
+    if (i + a.stages < a.steps) issue(i + a.stages);
+  }
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_measure_tma_stream(const void* buf, size_t bytes, int boxes, int stages, int contiguous,
+                                               int warps, int steps, int32_t* err, size_t* bytes_moved,
+                                               moe_stream_t stream) {
+  const size_t row_bytes = static_cast<size_t>(kPanelCols) * 2;
+  const size_t rows = bytes / row_bytes;
+  if (buf == nullptr || (reinterpret_cast<uintptr_t>(buf) & 15u) != 0 || rows < kPanelRows) return MOE_ERR_INVALID_ARG;
+  if (boxes < 1 || boxes > 3 || stages < 2 || stages > kMaxStages || steps < 1) return MOE_ERR_INVALID_ARG;
+  if (warps < 1 || warps > 4 || stages % warps != 0) return MOE_ERR_INVALID_ARG;
+  const uint32_t ring = kBox * static_cast<uint32_t>(boxes * stages);
+  if (ring > kMaxRing) return MOE_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return MOE_ERR_CUDA;
+  CUtensorMap map;
+  if (!moe::encode_map_bf16(&map, buf, rows, kPanelCols, kPanelRows)) return MOE_ERR_CUDA;
+  const size_t smem = ring + 1024;
+  if (cudaFuncSetAttribute(tma_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  TmaStreamArgs a{static_cast<const uint8_t*>(buf), static_cast<long long>(rows / kPanelRows), boxes, stages,
+                  contiguous != 0, warps, steps, err};
+  tma_stream_kernel<<<sms, 32 * warps, smem, static_cast<cudaStream_t>(stream)>>>(map, a);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (bytes_moved != nullptr) *bytes_moved = static_cast<size_t>(sms) * steps * boxes * kBox;
+  return MOE_OK;
 }

@@ -126,6 +126,32 @@ def test_device_error_rejects_null():
     assert moe.library().moe_get_device_error(None, None, ctypes.byref(code)) == 1
 
 
+def test_measure_calls_reject_bad_arguments():
+    L = moe.library()
+    panel = 128 * 7168 * 2  # one 128-row panel of the stream's [rows, 7168] bf16 view
+    moved = ctypes.c_size_t(0)
+
+    def tma(buf, nbytes, boxes, stages, steps, warps=1):
+        return L.moe_measure_tma_stream(buf, nbytes, boxes, stages, 0, warps, steps, None, ctypes.byref(moved),
+                                        None)
+
+    assert tma(None, panel, 2, 5, 10) == 1
+    assert tma(FAKE_MIS, panel, 2, 5, 10) == 1
+    assert tma(FAKE, panel - 1, 2, 5, 10) == 1      # under one panel
+    assert tma(FAKE, panel, 0, 5, 10) == 1          # boxes outside 1..3
+    assert tma(FAKE, panel, 4, 2, 10) == 1
+    assert tma(FAKE, panel, 1, 1, 10) == 1          # stages outside 2..16
+    assert tma(FAKE, panel, 1, 17, 10) == 1
+    assert tma(FAKE, panel, 3, 5, 10) == 1          # 240 KB ring: above 192 KB
+    assert tma(FAKE, panel, 2, 5, 0) == 1           # no steps
+    assert tma(FAKE, panel, 2, 4, 10, warps=0) == 1  # warps outside 1..4
+    assert tma(FAKE, panel, 1, 8, 10, warps=5) == 1
+    assert tma(FAKE, panel, 2, 5, 10, warps=2) == 1  # stages not a multiple of warps
+    assert moved.value == 0
+    assert L.moe_measure_hbm_read(None, 1024, None, None) == 1
+    assert L.moe_measure_hbm_read(FAKE, 1000, None, None) == 1
+
+
 def test_selftest_rejects_bad_arguments():
     L = moe.library()
     assert L.moe_selftest_wait_timeout(None, 1000, None) == 1
