@@ -30,15 +30,16 @@ TRACE_LIB = os.path.join(PKG, "libmoe_b200_trace.so")
 
 def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
           trace: bool = False) -> str:
-    """Compile the library; trace=True builds the timeline variant of the 2-SM pair GEMMs instead
-    (-DMOE_PAIR_TRACE, into libmoe_b200_trace.so; see pair_trace.py), never loaded by the package."""
+    """Compile the library; trace=True builds the timeline variant instead (-DMOE_PAIR_TRACE for the
+    2-SM pair GEMMs, -DMOE_LAYER_TRACE for the single-launch layer, into libmoe_b200_trace.so; see
+    pair_trace.py and layer_trace.py), never loaded by the package."""
     build_dir = BUILD + ("_trace" if trace else "")
     lib = TRACE_LIB if trace else LIB
     os.makedirs(build_dir, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     inc = os.path.join(ROOT, "include")
     headers += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
-    flags = FLAGS + (["-DMOE_PAIR_TRACE"] if trace else []) + (extra_flags or [])
+    flags = FLAGS + (["-DMOE_PAIR_TRACE", "-DMOE_LAYER_TRACE"] if trace else []) + (extra_flags or [])
     jobs = []
     objs = []
     for src in SOURCES:

@@ -195,12 +195,6 @@ moe_status_t check_plan(const moe_plan_t* p) {
   return MOE_OK;
 }
 
-moe_status_t check_bf16_weights(const moe_weights_t* w) {
-  if (w == nullptr) return MOE_ERR_INVALID_ARG;
-  if (w->dtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
-  return MOE_OK;
-}
-
 moe_status_t check_weights(const moe_weights_t* w, const moe_shape_t& s) {
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
   if (w->dtype != MOE_W_BF16 && w->dtype != MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;

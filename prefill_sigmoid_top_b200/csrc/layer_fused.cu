@@ -55,6 +55,39 @@
 namespace moe {
 namespace {
 
+// Phase timeline of the launch, per CTA (timeline build only, -DMOE_LAYER_TRACE; see layer_trace.py):
+// global-timer stamps (ns) of fixed points, the producer's total waits, and tile counts.
+enum LayerTraceSlot {
+  kLtStart = 0,         // kernel entry
+  kLtBarrier = 1,       // the grid barrier after the router logits passed
+  kLtPlan = 2,          // top-k and plan done, roles start
+  kLtFirstDown = 3,     // the producer claimed its first down tile
+  kLtLastUpPub = 4,     // this CTA published its last up tile
+  kLtLastDownPub = 5,   // this CTA published its last down tile
+  kLtFinStart = 6,      // first finalize item began (all y rows ready)
+  kLtFinEnd = 7,        // last finalize item ended
+  kLtWaitRows = 8,      // total ns the producer waited for an expert's h rows
+  kLtWaitSlot = 9,      // total ns the producer waited for a free ring slot
+  kLtUpTiles = 10,      // up tiles this CTA's epilogue finished
+  kLtDownTiles = 11,    // down tiles
+  kLtEnd = 12,          // kernel exit
+  kLtSlots = 16
+};
+#ifdef MOE_LAYER_TRACE
+constexpr int kLtCtas = 1024;
+__device__ unsigned long long g_layer_trace[kLtCtas][kLtSlots];
+#define MOE_LT(slot) g_layer_trace[blockIdx.x < kLtCtas ? blockIdx.x : kLtCtas - 1][(slot)]
+#define MOE_LT_SET(slot, v) (MOE_LT(slot) = (v))
+#define MOE_LT_FIRST(slot, v) (MOE_LT(slot) = MOE_LT(slot) ? MOE_LT(slot) : (v))
+#define MOE_LT_ADD(slot, v) (MOE_LT(slot) += (v))
+#define MOE_LT_NOW() global_timer_ns()
+#else
+#define MOE_LT_SET(slot, v) ((void)0)
+#define MOE_LT_FIRST(slot, v) ((void)0)
+#define MOE_LT_ADD(slot, v) ((void)0)
+#define MOE_LT_NOW() 0ull
+#endif
+
 constexpr int kThreads = 192;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBM = 128;                     // weight rows per tile (MMA M)
@@ -192,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto cnt = [&](int e) -> int { return offc[e + 1] - offc[e]; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) MOE_LT_SET(kLtStart, MOE_LT_NOW());
   unsigned* bar_word = args.sync;
   unsigned* next_work = args.sync + 1;
   unsigned* down_done = args.sync + 2;
@@ -275,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
       set_error(args.err, kErrTimeout);
     }
+    MOE_LT_SET(kLtBarrier, MOE_LT_NOW());
   }
   __syncthreads();
   if (*abort_flag) return;  // before any asynchronous work
@@ -473,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ producer
     if (lane == 0) {
+      MOE_LT_SET(kLtPlan, MOE_LT_NOW());
       prefetch_tensor_map(&tm_gate);
       prefetch_tensor_map(&tm_up);
       prefetch_tensor_map(&tm_down);
@@ -526,6 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const bool up = w.x == kKindUp;
       const int e = w.y, wt = w.z, lt = w.w;
+      if (!up && lane == 0) MOE_LT_FIRST(kLtFirstDown, MOE_LT_NOW());
       const int nrows = min(kNmax, cnt(e) - lt * kNmax);
       const int N = (nrows + 15) & ~15;
       const int row0 = offp[e] + lt * kNmax;
@@ -554,7 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // half issued
         bool dep = true;
         if (lane == 0) {
+          [[maybe_unused]] const unsigned long long t0 = MOE_LT_NOW();
           dep = wait_count(up_done + e, static_cast<unsigned>(Wu * (tp[e + 1] - tp[e])), abort_flag);
+          MOE_LT_ADD(kLtWaitRows, MOE_LT_NOW() - t0);
           if (dep) {
             fence_proxy_async_global();
           } else {
@@ -567,7 +606,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int step = 0; step < nsteps; ++step, ++it) {
         const int s = it % kSlots;
         bool fs = true;
-        if (lane == 0) fs = mbar_wait_bounded(&empty[s], ((it / kSlots) & 1) ^ 1, abort_flag);
+        if (lane == 0) {
+          [[maybe_unused]] const unsigned long long t0 = MOE_LT_NOW();
+          fs = mbar_wait_bounded(&empty[s], ((it / kSlots) & 1) ^ 1, abort_flag);
+          MOE_LT_ADD(kLtWaitSlot, MOE_LT_NOW() - t0);
+        }
         fs = __shfl_sync(0xffffffffu, fs, 0);
         if (!fs) {
           if (lane == 0) {
@@ -702,6 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *abort_flag = 1;
             set_error(args.err, kErrTimeout);
           }
+          MOE_LT_FIRST(kLtFinStart, MOE_LT_NOW());
           *epi_go = ready ? 1 : 0;
         }
         epi_sync();
@@ -793,7 +837,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4*>(args.residual_out + static_cast<size_t>(t) * H + p * 8) = r;
             }
           }
-          if (et == 0) mbar_arrive_one(fin_bar);
+          if (et == 0) {
+            MOE_LT_SET(kLtFinEnd, MOE_LT_NOW());
+            mbar_arrive_one(fin_bar);
+          }
           continue;
         }
         // The whole token: the many-token kernel's 256-thread CTA, virtual
@@ -876,7 +923,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(args.residual_out + static_cast<size_t>(t) * H + p * 8) = r;
           }
         }
-        if (et == 0) mbar_arrive_one(fin_bar);  // fin_w and part[] are free again (last epi_sync above)
+        if (et == 0) {
+          MOE_LT_SET(kLtFinEnd, MOE_LT_NOW());
+          mbar_arrive_one(fin_bar);  // fin_w and part[] are free again (last epi_sync above)
+        }
         continue;
       }
       // ---- a projection tile
@@ -945,6 +995,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (et == 0) {
         __threadfence();
         red_release_add(up ? up_done + e : down_done, 1u);
+        MOE_LT_SET(up ? kLtLastUpPub : kLtLastDownPub, MOE_LT_NOW());
+        MOE_LT_ADD(up ? kLtUpTiles : kLtDownTiles, 1ull);
       }
       ++ti;
     }
@@ -953,6 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (tid == 0) MOE_LT_SET(kLtEnd, MOE_LT_NOW());
 }
 
 }  // namespace
@@ -994,3 +1047,15 @@ cudaError_t launch_layer_fused(const CUtensorMap& w_gate, const CUtensorMap& w_u
 }
 
 }  // namespace moe
+
+#ifdef MOE_LAYER_TRACE
+// Host access to the phase timeline of the last single-launch layers (timeline build only).
+extern "C" __attribute__((visibility("default"))) int moe_layer_trace_read(void* host, size_t bytes) {
+  return cudaMemcpyFromSymbol(host, moe::g_layer_trace, bytes) == cudaSuccess ? 0 : 1;
+}
+extern "C" __attribute__((visibility("default"))) int moe_layer_trace_clear() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, moe::g_layer_trace) != cudaSuccess) return 1;
+  return cudaMemset(p, 0, sizeof(moe::g_layer_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
