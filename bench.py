@@ -45,9 +45,9 @@ DEFAULT_WORKLOADS = (1, 2, 3, 4)
 # the kernel sources hash to the recorded value; otherwise "traffic" is null.
 NCU_TRAFFIC = {
     # (workload, kernel): (DRAM bytes per launch, hash of the kernel's sources)
-    # decode M=8, the single-launch layer: E=32 capture (2.7368 GB read + write for 31 touched
-    # experts, 1.0020 x its 2.7312 GB of algorithmic bytes) scaled to 95 touched experts
-    (1, "layer_fused"): (8_386_900_000, "d815c00a1de4a117"),
+    # decode M=8, the single-launch layer, captured at full size, one pass (8.3777 GB read + 4.4 MB
+    # written, 1.0013 x its 8.3715 GB of algorithmic bytes)
+    (1, "layer_fused"): (8_382_036_224, "9c39ca834ce5fa81"),
     # batch M=512 and prefill M=2048: the up projection (2-SM pair kernel) captured at full size, one pass
     # (dram__bytes_read.sum + dram__bytes_write.sum of one launch)
     (2, "pair_up"): (15_305_074_944, "5c0cd642d8591f67"),
