@@ -239,6 +239,13 @@ bool want_pair_gather(const moe_shape_t& s) {
   return pair_nmax(s) == 128;
 }
 
+// Whether the layer routes through the screened path (router_screen.cu), with the y region of its
+// workspace as scratch.
+bool route_screens(const moe_shape_t& s) {
+  if (!moe::screen_eligible(s.M, s.H, s.E, s.top_k)) return false;
+  return moe::screen_scratch_bytes(s.M, s.H, s.E) <= static_cast<size_t>(s.M) * s.top_k * s.H * sizeof(uint16_t);
+}
+
 // Whether the up projection of this shape launches the x gather into plan order first.
 bool up_pregathers(const moe_shape_t& s) {
   if (!want_pregather(s)) return false;
@@ -580,9 +587,15 @@ moe_status_t run_layer_to_y(const moe_bf16_t* x, const moe_bf16_t* w_router, con
   auto* h = reinterpret_cast<moe_bf16_t*>(base + L.h);
   auto* y = reinterpret_cast<moe_bf16_t*>(base + L.y);
   float* logits = reinterpret_cast<float*>(base + L.logits);
-  if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
-    return st;
-  if ((st = cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, ids, tw, cs))) != MOE_OK) return st;
+  if (route_screens(s)) {  // its scratch: the y region, written only by the down projection
+    if ((st = cuda_status(moe::launch_route_screened(x, w_router, bias, s.M, s.H, s.E, s.top_k, base + L.y, ids,
+                                                     tw, err, cs))) != MOE_OK)
+      return st;
+  } else {
+    if ((st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs))) != MOE_OK)
+      return st;
+    if ((st = cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, ids, tw, cs))) != MOE_OK) return st;
+  }
   moe_plan_t plan{sorted, bexp, counts, offs, ntpp};
   if (want_self_route(s, w->dtype)) {
     if ((st = run_up_routed(x, w, ids, s, sorted, bexp, counts, offs, ntpp, h, err, cs)) != MOE_OK) return st;
@@ -609,6 +622,9 @@ moe_status_t run_layer_to_y(const moe_bf16_t* x, const moe_bf16_t* w_router, con
 namespace moe {
 bool encode_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   return make_map_bf16(map, base, rows, cols, box_rows);
+}
+bool encode_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols_bytes, uint32_t box_rows) {
+  return make_map_u8(map, base, rows, cols_bytes, box_rows);
 }
 
 int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,
@@ -643,7 +659,8 @@ size_t moe_align_capacity(moe_shape_t s) {
 
 size_t moe_route_workspace_size(moe_shape_t s) {
   if (check_shape(s) != MOE_OK) return 0;
-  return align_up(static_cast<size_t>(s.M) * s.E * sizeof(float));
+  const size_t logits = align_up(static_cast<size_t>(s.M) * s.E * sizeof(float));
+  return logits + (moe::screen_shape_ok(s.M, s.H, s.E, s.top_k) ? moe::screen_scratch_bytes(s.M, s.H, s.E) : 0);
 }
 
 size_t moe_up_workspace_size(moe_shape_t s, moe_wdtype_t dtype) {
@@ -666,6 +683,11 @@ moe_status_t moe_route(const moe_bf16_t* x, const moe_bf16_t* w_router, const fl
   if (!ws || ws_bytes < moe_route_workspace_size(s)) return MOE_ERR_WORKSPACE;
   auto cs = static_cast<cudaStream_t>(stream);
   float* logits = static_cast<float*>(ws);
+  if (moe::screen_eligible(s.M, s.H, s.E, s.top_k) && aligned16(ws)) {
+    uint8_t* scratch = static_cast<uint8_t*>(ws) + align_up(static_cast<size_t>(s.M) * s.E * sizeof(float));
+    return cuda_status(moe::launch_route_screened(x, w_router, bias, s.M, s.H, s.E, s.top_k, scratch, topk_ids,
+                                                  topk_w, nullptr, cs));
+  }
   st = cuda_status(moe::launch_router_logits(x, w_router, bias, s.M, s.H, s.E, logits, cs));
   if (st != MOE_OK) return st;
   return cuda_status(moe::launch_router_topk(logits, s.M, s.E, s.top_k, topk_ids, topk_w, cs));
@@ -843,11 +865,13 @@ moe_status_t moe_tp_layer(const moe_bf16_t* x, const moe_bf16_t* w_router, const
 
 int moe_layer_kernel_count(moe_shape_t s, moe_wdtype_t dtype) {
   if (check_shape(s) != MOE_OK || (dtype != MOE_W_BF16 && dtype != MOE_W_NVFP4)) return -1;
-  if (dtype == MOE_W_NVFP4)  // router x2, align, amax x, quantize x, gather tiles, up (+ amax h), quantize h, down, finalize
-    return 10;
-  if (want_fused_layer(s, dtype)) return 1;  // the whole layer in one launch
-  if (want_self_route(s, dtype)) return 5;   // router x2, up with the plan, down, finalize
-  return 6 + (up_pregathers(s) ? 1 : 0);    // router x2, align, [gather x], up, down, finalize
+  // routing: logits + top-k, or screened: digits, integer partial logits, candidates + exact logits + top-k
+  const int route = route_screens(s) ? 3 : 2;
+  if (dtype == MOE_W_NVFP4)  // routing, align, amax x, quantize x, gather tiles, up (+ amax h), quantize h, down, finalize
+    return route + 8;
+  if (want_fused_layer(s, dtype)) return 1;      // the whole layer in one launch
+  if (want_self_route(s, dtype)) return route + 3;  // routing, up with the plan, down, finalize
+  return route + 4 + (up_pregathers(s) ? 1 : 0);   // routing, align, [gather x], up, down, finalize
 }
 
 moe_status_t moe_quantize_nvfp4(const moe_bf16_t* src, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* codes,

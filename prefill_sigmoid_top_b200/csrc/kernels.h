@@ -13,6 +13,17 @@ namespace moe {
 // api.cu: validation of moe_route's arguments (a moe_status_t value).
 // 2-D bf16 tensor map [rows, cols] with boxes of box_rows x 64 elements and the 128-byte swizzle.
 bool encode_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// 2-D byte tensor map [rows, cols_bytes] with boxes of box_rows x 128 bytes and the 128-byte swizzle.
+bool encode_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols_bytes, uint32_t box_rows);
+
+// router_screen.cu: routing of many tokens from exact canonical logits of the candidate experts only
+// (the same ids and weights as launch_router_logits + launch_router_topk).
+bool screen_shape_ok(int M, int H, int E, int K);   // shapes it takes (sizes the workspaces)
+bool screen_eligible(int M, int H, int E, int K);   // shapes it takes, unless MOE_ROUTER_SCREEN=0
+size_t screen_scratch_bytes(int M, int H, int E);   // device scratch it needs (16-byte aligned base)
+cudaError_t launch_route_screened(const uint16_t* x, const uint16_t* w_router, const float* bias, int M, int H, int E,
+                                  int K, uint8_t* scratch, int32_t* topk_ids, float* topk_w, int32_t* err,
+                                  cudaStream_t stream);
 
 int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,
                      const void* topk_w);

@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "router_dot.cuh"
+#include "router_select.cuh"
 
 namespace moe {
 namespace {
@@ -167,15 +168,6 @@ cudaError_t launch_staged(const uint16_t* x, const uint16_t* w_router, const flo
   return cudaGetLastError();
 }
 
-// (value, id) ordering of the selection: larger value first, then lower id.
-__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
-}
-
-// A NaN logit enters the selection (and its score) as -inf: it ranks below
-// every other logit, so a selected id always lies in [0, E).
-__device__ __forceinline__ float selection_key(float z) { return isnan(z) ? -INFINITY : z; }
-
 template <int kPerLane>
 __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restrict__ logits, int M, int E, int K,
                                                           int32_t* __restrict__ topk_ids,
@@ -183,50 +175,9 @@ __global__ void __launch_bounds__(128) router_topk_kernel(const float* __restric
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (t >= M) return;
-  float v[kPerLane];
-  bool live[kPerLane];
-#pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    const int e = lane + 32 * i;
-    live[i] = e < E;
-    v[i] = live[i] ? selection_key(logits[static_cast<size_t>(t) * E + e]) : -INFINITY;
-  }
-  float sel_v = 0.0f;
-  int sel_id = 0;
-  for (int k = 0; k < K; ++k) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i)
-      if (live[i] && better(v[i], lane + 32 * i, bv, bi)) {
-        bv = v[i];
-        bi = lane + 32 * i;
-      }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (better(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kPerLane; ++i)  // the owner retires the winner
-      if (lane + 32 * i == bi) live[i] = false;
-    if (lane == k) {
-      sel_v = bv;
-      sel_id = bi;
-    }
-  }
-  const float s = (lane < K) ? 1.0f / (1.0f + expf(-sel_v)) : 0.0f;
-  float total = s;
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
-  if (lane < K) {
-    topk_ids[static_cast<size_t>(t) * K + lane] = sel_id;
-    topk_w[static_cast<size_t>(t) * K + lane] = s / total;
-  }
+  const float* zt = logits + static_cast<size_t>(t) * E;
+  topk_sigmoid_token<kPerLane>([&](int e) { return zt[e]; }, E, K, lane, topk_ids + static_cast<size_t>(t) * K,
+                               topk_w + static_cast<size_t>(t) * K);
 }
 
 template <int kPerLane>

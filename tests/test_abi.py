@@ -197,12 +197,19 @@ def test_layer_kernel_count(monkeypatch):
     monkeypatch.delenv("MOE_FUSED_LAYER")
     many_experts = moe.Shape(M=2, H=7168, I=2048, E=512, top_k=8, block_size=16)
     assert moe.layer_kernel_count(many_experts) == 5  # the single launch takes E <= 256
+    # from 128 tokens the routing is screened: digits, integer partial logits, then one kernel for the
+    # candidates, their exact logits and the top-k
     batch = moe.Shape(M=512, H=7168, I=2048, E=256, top_k=16, block_size=64)
-    assert moe.layer_kernel_count(batch) == 6         # align; the up kernel gathers x rows itself
+    assert moe.layer_kernel_count(batch) == 7         # routing 3, align; the up kernel gathers x rows itself
     prefill = moe.Shape(M=2048, H=7168, I=2048, E=256, top_k=16, block_size=128)
-    assert moe.layer_kernel_count(prefill) == 7       # align and a gather pass of x (256-row token tiles)
+    assert moe.layer_kernel_count(prefill) == 8       # routing 3, align and a gather pass of x (256-row tiles)
     monkeypatch.setenv("MOE_PAIR_GATHER", "0")
-    assert moe.layer_kernel_count(batch) == 7
+    assert moe.layer_kernel_count(batch) == 8
     monkeypatch.delenv("MOE_PAIR_GATHER")
+    assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 11
+    monkeypatch.setenv("MOE_ROUTER_SCREEN", "0")      # logits of every expert + top-k
+    assert moe.layer_kernel_count(batch) == 6
+    assert moe.layer_kernel_count(prefill) == 7
     assert moe.layer_kernel_count(batch, moe.MOE_W_NVFP4) == 10
+    monkeypatch.delenv("MOE_ROUTER_SCREEN")
     assert moe.layer_kernel_count(moe.Shape(M=16, H=255, I=128, E=8, top_k=2, block_size=16)) == -1
