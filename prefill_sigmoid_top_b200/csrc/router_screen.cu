@@ -57,23 +57,31 @@ struct RowStats {
 static_assert(sizeof(RowStats) == 64, "row stats");
 
 // ---------------------------------------------------------------------------- 1. digits and bounds
-__global__ void __launch_bounds__(128) screen_quantize_kernel(const uint16_t* __restrict__ x,
-                                                              const uint16_t* __restrict__ w, int M, int E, int H,
-                                                              int8_t* __restrict__ hi, int8_t* __restrict__ lo,
-                                                              RowStats* __restrict__ stats) {
-  extern __shared__ __align__(16) uint8_t qsm[];  // [4][H] bf16: each warp's row, read from global once
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 4 + warp;
-  if (row >= M + E) return;  // uniform per warp; no block-wide barrier follows
+constexpr int kQThreads = 128;                  // one CTA per row
+constexpr int kQPer = 8;                        // 16-byte chunks per thread (H <= 8192)
+
+__global__ void __launch_bounds__(kQThreads) screen_quantize_kernel(const uint16_t* __restrict__ x,
+                                                                    const uint16_t* __restrict__ w, int M, int E,
+                                                                    int H, int8_t* __restrict__ hi,
+                                                                    int8_t* __restrict__ lo,
+                                                                    RowStats* __restrict__ stats) {
+  __shared__ float red_f[kQThreads / 32];
+  __shared__ int red_i[kQThreads / 32];
+  __shared__ long long red_l[kQThreads / 32];
+  const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint16_t* src = row < M ? x + static_cast<size_t>(row) * H : w + static_cast<size_t>(row - M) * H;
-  uint4* rs = reinterpret_cast<uint4*>(qsm + static_cast<size_t>(warp) * H * 2);
   const int nc = H / 8;
+  uint4 v[kQPer];  // chunks tid, tid + 128, ... of the row, read once
   float m = 0.0f;
   bool fin = true;
-  for (int c = lane; c < nc; c += 32) {
-    const uint4 v = *reinterpret_cast<const uint4*>(src + c * 8);
-    rs[c] = v;
-    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < kQPer; ++k) {
+    const int c = tid + kQThreads * k;
+    v[k] = c < nc ? *reinterpret_cast<const uint4*>(src + c * 8) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int k = 0; k < kQPer; ++k) {
+    const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float a = bf16_lo(wd[i]), b = bf16_hi(wd[i]);
@@ -83,7 +91,20 @@ __global__ void __launch_bounds__(128) screen_quantize_kernel(const uint16_t* __
   }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  fin = __all_sync(0xffffffffu, fin);  // (each lane reads back below only the chunks it wrote)
+  const int wfin = __all_sync(0xffffffffu, fin) ? 1 : 0;
+  if (lane == 0) {
+    red_f[warp] = m;
+    red_i[warp] = wfin;
+  }
+  __syncthreads();
+  m = 0.0f;
+  fin = true;
+#pragma unroll
+  for (int q = 0; q < kQThreads / 32; ++q) {
+    m = fmaxf(m, red_f[q]);
+    fin = fin && red_i[q] != 0;
+  }
+  __syncthreads();  // red_* are reused below
   int ex = 0;
   frexpf(m, &ex);  // m = f * 2^ex, f in [0.5, 1) (m = 0: ex = 0)
   // s = 2^(ex - 13) as a float needs ex - 13 >= -149 and 1/s needs 13 - ex <= 127; a row that misses
@@ -96,9 +117,11 @@ __global__ void __launch_bounds__(128) screen_quantize_kernel(const uint16_t* __
   long long nx2 = 0;
   int8_t* hrow = hi + static_cast<size_t>(row) * H;
   int8_t* lrow = lo + static_cast<size_t>(row) * H;
-  for (int c = lane; c < nc; c += 32) {
-    const uint4 v = rs[c];
-    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < kQPer; ++k) {
+    const int c = tid + kQThreads * k;
+    if (c >= nc) break;
+    const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
     uint32_t hpk[2] = {0u, 0u}, lpk[2] = {0u, 0u};
     int sq = 0;
 #pragma unroll
@@ -126,6 +149,21 @@ __global__ void __launch_bounds__(128) screen_quantize_kernel(const uint16_t* __
     nx2 += __shfl_xor_sync(0xffffffffu, nx2, off);
   }
   if (lane == 0) {
+    red_f[warp] = eps;
+    red_i[warp] = nh;
+    red_l[warp] = nx2;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    eps = 0.0f;
+    nh = 0;
+    nx2 = 0;
+#pragma unroll
+    for (int q = 0; q < kQThreads / 32; ++q) {
+      eps = fmaxf(eps, red_f[q]);
+      nh += red_i[q];
+      nx2 += red_l[q];
+    }
     RowStats st;
     const double sd = s, ed = eps;
     st.s = sd;
@@ -268,9 +306,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
     if (!ok) {
       if (lane == 0) set_error(a.err, kErrTimeout);
     } else {
-      const int t = t0 + q * 32 + lane;
+      // lane = token of this warp's 32; each 16-column block goes through shared memory (the ring is
+      // idle once the accumulators are complete) so that the stores are 128-byte runs of one token's row
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      double* out = a.partial + (static_cast<size_t>(blockIdx.z) * a.M + (t < a.M ? t : 0)) * a.E;
+      double* stage = reinterpret_cast<double*>(ring) + (warp - 2) * 32 * 17;  // [32 tokens][16 + 1]
+      const int half = lane >> 4, col = lane & 15;
 #pragma unroll 1
       for (int cb = 0; cb < kSBN; cb += 16) {
         uint32_t hh[16], hl[16], ll[16];
@@ -278,15 +318,19 @@ __global__ void __launch_bounds__(kSThreads, 1)
         tmem_load_16(lane_base + kSBN + cb, hl);
         tmem_load_16(lane_base + 2 * kSBN + cb, ll);
         tmem_load_wait();
-        if (t < a.M) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int e = e0 + cb + j;
-            if (e < a.E)
-              out[e] = 16384.0 * static_cast<int32_t>(hh[j]) + 128.0 * static_cast<int32_t>(hl[j]) +
-                       static_cast<double>(static_cast<int32_t>(ll[j]));  // exact: an integer below 2^53
-          }
+        for (int j = 0; j < 16; ++j)  // exact: an integer below 2^53
+          stage[lane * 17 + j] = 16384.0 * static_cast<int32_t>(hh[j]) + 128.0 * static_cast<int32_t>(hl[j]) +
+                                 static_cast<double>(static_cast<int32_t>(ll[j]));
+        __syncwarp();
+        const int e = e0 + cb + col;
+#pragma unroll 4
+        for (int r = half; r < 32; r += 2) {  // two tokens' 16 columns per store instruction
+          const int t = t0 + q * 32 + r;
+          if (t < a.M && e < a.E)
+            a.partial[(static_cast<size_t>(blockIdx.z) * a.M + t) * a.E + e] = stage[r * 17 + col];
         }
+        __syncwarp();
       }
     }
   }
@@ -326,6 +370,7 @@ __global__ void __launch_bounds__(128) screen_route_kernel(const uint16_t* __res
     double p[kPer];  // exact sums of integers below 2^53, all loads of a slice in flight together
 #pragma unroll
     for (int i = 0; i < kPer; ++i) p[i] = 0.0;
+#pragma unroll 4
     for (int sl = 0; sl < slices; ++sl) {
       const double* ps = partial + (static_cast<size_t>(sl) * M + t) * E + lane;
 #pragma unroll
@@ -529,14 +574,9 @@ cudaError_t launch_route_screened(const uint16_t* x, const uint16_t* w_router, c
   auto* partial = reinterpret_cast<double*>(scratch + L.partial);
   const int R = M + E;
 
-  const int qsmem = 4 * H * 2;
-  cudaError_t st = cudaSuccess;
-  if (qsmem > 48 * 1024 &&
-      (st = cudaFuncSetAttribute(screen_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qsmem)) !=
-          cudaSuccess)
-    return st;
-  screen_quantize_kernel<<<(R + 3) / 4, 128, qsmem, stream>>>(x, w_router, M, E, H, hi, lo, stats);
-  if ((st = cudaGetLastError()) != cudaSuccess) return st;
+  screen_quantize_kernel<<<R, kQThreads, 0, stream>>>(x, w_router, M, E, H, hi, lo, stats);
+  cudaError_t st = cudaGetLastError();
+  if (st != cudaSuccess) return st;
 
   // digit planes as [rows, H] int8 tensors read in 128-byte-wide boxes with the 128-byte swizzle
   CUtensorMap mxh, mxl, mwh, mwl;
