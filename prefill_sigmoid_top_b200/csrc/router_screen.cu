@@ -19,7 +19,8 @@
 //       fp32 logit z, from  |x.w - s_x s_w P| <= eps_x s_w sum|X_w| + eps_w sum|x|  and the error of the
 //       canonical fp32 sum,  |z - (x.w + b)| <= g_n (||x|| ||w|| + |b|) + n 2^-149  (n = H/32 + 6 roundings
 //       of a sum of products of bf16 values, the last term for underflow; sum |x_h w_h| <= ||x|| ||w||),
-//       plus margins for the fp64 arithmetic of the bound itself;
+//       plus margins for the fp64 arithmetic of the bound itself (valid while ||x|| ||w|| + |b| < 2^120,
+//       so that no fp32 sum of the canonical order overflows; otherwise the pair is a candidate);
 //     - with A the K experts of largest za and L = min over A of (za - d), an expert whose za + d < L
 //       has z < L <= z of each of the K experts of A, so it cannot be selected: the others (at least the
 //       K of A) are the candidates; a row that is not finite makes all its pairs candidates;
@@ -387,7 +388,9 @@ __global__ void __launch_bounds__(128) screen_route_kernel(const uint16_t* __res
       if (e >= E) continue;
       const RowStats ws = stats[M + e];
       const double b = bias != nullptr ? static_cast<double>(bias[e]) : 0.0;
-      if (xst.finite != 0.0 && ws.finite != 0.0 && isfinite(b)) {
+      // the bound below holds while no fp32 sum of the canonical order can overflow: every partial sum is
+      // at most sum |x_h w_h| + |b| <= ||x|| ||w|| + |b| (times 1 + g_n), far below 2^128 under 2^120
+      if (xst.finite != 0.0 && ws.finite != 0.0 && isfinite(b) && xst.n2 * ws.n2 + fabs(b) < 0x1p120) {
         const double z = xst.s * ws.s * p[i] + b;
         double d = xst.eps * ws.nhat1 + ws.eps * xst.n1 + gam * (xst.n2 * ws.n2 + fabs(b)) + under;
         d = d * (1.0 + 1e-9) + fabs(z) * 0x1p-50;

@@ -81,7 +81,7 @@ def test_rows_that_are_not_finite(monkeypatch):
     _check(x, w_r, b, K, monkeypatch)
 
 
-@pytest.mark.parametrize("scale", [2.0 ** -60, 2.0 ** 40])
+@pytest.mark.parametrize("scale", [2.0 ** -60, 2.0 ** 40, 2.0 ** 125])  # 2^125: canonical fp32 sums overflow
 def test_magnitudes_far_from_one(scale, monkeypatch):
     M, H, E, K = 144, 512, 48, 6
     cfg = inputs.WORKLOADS[0].with_(M=M, H=H, E=E, K=K, bias="normal", seed=5)
