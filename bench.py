@@ -815,6 +815,14 @@ TMA_PROBES = [(1, 10, False, 1), (2, 5, False, 1), (3, 4, False, 1), (1, 10, Tru
               (3, 4, True, 1), (2, 6, False, 2), (2, 4, False, 4), (3, 4, False, 4)]
 
 
+# the copy mixes of moe_measure_tma_mix: what a k-step copies besides its two 16 KB code boxes
+TMA_MIXES = {0: "code boxes only",
+             1: "+ 8 KB token box (second warp)",
+             2: "+ token box and three 2 KB scale chunks, all four from the second warp (the NVFP4 kernels' stage)",
+             3: "+ token box and three 2 KB scale chunks, one of them from the first warp",
+             4: "+ token box; every fourth step three 8 KB chunks (the scales of four steps)"}
+
+
 def run_probe_tma(args):
     """The weight-panel stream of the grouped GEMMs on its own: one CTA per SM copying 128 x 64 bf16 boxes
     of 128-row panels into a ring of shared-memory stages (moe_measure_tma_stream), from an 8 GB buffer
@@ -849,13 +857,25 @@ def run_probe_tma(args):
                          "copy": "bulk 16 KB (panel stored box by box)" if contiguous else "2-D tensor box 128 x 64",
                          "in_flight_kb_per_sm": boxes * stages * 16, "GBps": moved / sec / 1e9,
                          "us_per_stage": sec * 1e6 / steps})
+    mixes = []
+    for mix in TMA_MIXES:
+        per_step = {0: 32768, 1: 40960, 2: 47104, 3: 47104, 4: 47104}[mix]
+        steps = int((4 << 30) / (148 * per_step))
+        moved, sec = timed(lambda: moe.measure_tma_mix(buf, mix, 4, steps, err))
+        mixes.append({"mix": mix, "copies": TMA_MIXES[mix], "stages": 4, "GBps": moved / sec / 1e9,
+                      "us_per_step": sec * 1e6 / steps})
     if moe.get_device_error(err) != 0:
-        raise RuntimeError("moe_measure_tma_stream: a bounded wait expired")
+        raise RuntimeError("moe_measure_tma_stream / moe_measure_tma_mix: a bounded wait expired")
     read_gbs = measure_read_ceiling(moe, torch, buf)
     print(json.dumps({"kernel": "tma_stream_kernel (moe_measure_tma_stream)",
                       "ctas": "one per SM; one thread per issuing warp waits and issues",
                       "panel": "128 rows x 7168 bf16 columns, 64-column steps", "hbm_read_ceiling_gbs": read_gbs,
                       "probes": rows}), flush=True)
+    print(json.dumps({"kernel": "tma_mix_kernel (moe_measure_tma_mix)",
+                      "ctas": "one per SM; the first lanes of two warps issue",
+                      "step": "one k-step of 256 e2m1 elements: two 128 x 128-byte code boxes (32 KB) from HBM, "
+                              "token rows from L2, scale chunks from HBM",
+                      "mixes": mixes}), flush=True)
 
 
 def main(argv=None):

@@ -53,6 +53,33 @@ MOE_API moe_status_t moe_measure_tma_stream(const void* buf, size_t bytes, int b
                                             int warps, int steps, int32_t* err, size_t* bytes_moved,
                                             moe_stream_t stream);
 
+/* The copy mix of one stage of the NVFP4 GEMMs, without the GEMM: one CTA per
+ * SM, two issuing warps, copies into a ring of `stages` (2..4) shared-memory
+ * slots that are discarded, so that the rate of a stage's copies can be
+ * measured against their mix.
+ *
+ * buf (16-byte aligned, at least 256 MB) is split in two.  Its first 7/8 is a
+ * byte matrix [rows, 3584] (e2m1 codes of weight rows of 7168 elements) cut
+ * into panels of 128 rows; its first 8192 rows (28 MB, which stay in L2) also
+ * serve as token rows.  Its last 1/8 holds 2 KB scale chunks.  A step is one
+ * k-step of 256 elements: the first warp copies two code boxes of 128 rows x
+ * 128 bytes (32 KB, 128-byte swizzle) from two panels; what else a step holds
+ * is `mix`:
+ *   0  nothing (the code boxes alone);
+ *   1  a box of 64 token rows x 128 bytes (8 KB), copied by the second warp;
+ *   2  the token box and three 2 KB scale chunks, all four copied by the
+ *      second warp (the copies of a stage of the NVFP4 kernels);
+ *   3  the same bytes, one scale chunk copied by the first warp;
+ *   4  the token box, and on every fourth step three 8 KB chunks (the scales
+ *      of four k-steps in one copy each), copied by the second warp.
+ * `steps` (>= 8) steps per CTA.  *bytes_moved (host, nullable) receives the
+ * bytes one call copies; time the call with events on `stream`.  err (device
+ * int32, nullable) gets MOE_ERR_TIMEOUT if a copy did not land within the
+ * bounded wait.  INVALID_ARG for a null or misaligned buffer, a buffer under
+ * 256 MB, or mix / stages / steps outside the ranges above. */
+MOE_API moe_status_t moe_measure_tma_mix(const void* buf, size_t bytes, int mix, int stages, int steps, int32_t* err,
+                                         size_t* bytes_moved, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

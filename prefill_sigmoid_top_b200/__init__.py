@@ -117,6 +117,8 @@ def _declare(L):
         "moe_measure_hbm_read": (st, [vp, sz, vp, vp]),
         "moe_measure_tma_stream": (st, [vp, sz, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, vp, ctypes.POINTER(ctypes.c_size_t), vp]),
+        "moe_measure_tma_mix": (st, [vp, sz, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp,
+                                     ctypes.POINTER(ctypes.c_size_t), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -479,6 +481,18 @@ def measure_tma_stream(buf, boxes: int, stages: int, contiguous: bool, steps: in
                                             1 if contiguous else 0, int(warps), int(steps),
                                             _ptr(err_flag) if err_flag is not None else None,
                                             ctypes.byref(moved), _stream()), "moe_measure_tma_stream")
+    return int(moved.value)
+
+
+def measure_tma_mix(buf, mix: int, stages: int, steps: int, err_flag=None) -> int:
+    """Enqueue one stream of the NVFP4 GEMMs' stage copy mix ``mix`` over the tensor ``buf``
+    (moe_measure_tma_mix: ``stages`` slots in flight, ``steps`` k-steps per CTA); returns the bytes the call
+    copies into shared memory."""
+    _need_cuda(buf)
+    moved = ctypes.c_size_t(0)
+    _check(library().moe_measure_tma_mix(_ptr(buf), buf.numel() * buf.element_size(), int(mix), int(stages),
+                                         int(steps), _ptr(err_flag) if err_flag is not None else None,
+                                         ctypes.byref(moved), _stream()), "moe_measure_tma_mix")
     return int(moved.value)
 
 

@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 SOURCES = ["api.cu", "router.cu", "router_screen.cu", "align.cu", "finalize.cu", "gemm_bf16.cu", "gemm_persistent.cu",
-           "gemm_pair.cu", "nvfp4.cu", "layer_fused.cu", "measure.cu", "tp_finalize.cu"]
+           "gemm_pair.cu", "nvfp4.cu", "nvfp4_pair.cu", "layer_fused.cu", "measure.cu", "tp_finalize.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-DNDEBUG", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include"), "-I", CSRC]

@@ -84,6 +84,22 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
+// NVFP4 scale atoms ([blocks][kdim/64][512 bytes]) as a 2-D byte tensor of
+// 256-byte rows, read in boxes of 8 rows (one stage's four atoms, 2 KB) with
+// no swizzle: the shared-memory copy is the global bytes in order.
+bool make_map_sf(CUtensorMap* map, const void* base, uint64_t bytes, uint32_t box_rows = 8) {
+  auto fn = encode_fn();
+  if (fn == nullptr || bytes % (256 * box_rows) != 0) return false;
+  cuuint64_t dims[2] = {256, bytes / 256};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {256, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Token-tile width of the single-SM grouped kernels, from the mean routed rows
 // per expert (known on the host without reading the plan back): decode shapes
 // (<= 24) use 32-row tiles, larger ones 128-row tiles (which also selects the
@@ -430,6 +446,15 @@ moe_status_t run_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_pla
 
 int num_sms();
 
+// Whether the NVFP4 projections run on 2-SM pairs (nvfp4_pair.cu): whenever the weight blocks of a pair
+// divide the expert (up: I a multiple of 256, down: H a multiple of 512).  MOE_NVFP4_PAIR=0 keeps the
+// single-SM kernels (the tests cover both).
+bool want_nvfp4_pair(const moe_shape_t& s, bool up) {
+  if (const char* env = std::getenv("MOE_NVFP4_PAIR"))
+    if (std::strcmp(env, "0") == 0) return false;
+  return up ? s.I % 256 == 0 : s.H % 512 == 0;
+}
+
 moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
                           const moe_shape_t& s, moe_bf16_t* h, void* ws, int32_t* err, cudaStream_t stream,
                           unsigned* h_amax) {
@@ -469,6 +494,14 @@ moe_status_t run_up_nvfp4(const moe_bf16_t* x, const moe_weights_t* w, const moe
   a.gs_a1 = w->up_gs;
   a.act_amax = amax;
   a.out_amax = h_amax;
+  if (want_nvfp4_pair(s, true)) {
+    CUtensorMap sg, su, sx;
+    const uint64_t wsf = static_cast<uint64_t>(s.E) * (s.I / 128) * (s.H / 64) * 512;
+    if (!make_map_sf(&sg, a.sfa0, wsf) || !make_map_sf(&su, a.sfa1, wsf) ||
+        !make_map_sf(&sx, a.sfb, static_cast<uint64_t>(tiles) * (s.H / 64) * 512))
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_nvfp4_pair_up(mg, mu, mx, sg, su, sx, a, num_sms(), stream));
+  }
   return cuda_status(moe::launch_nvfp4_up(mg, mu, mx, a, num_sms(), stream));
 }
 
@@ -510,6 +543,13 @@ moe_status_t run_down_nvfp4(const moe_bf16_t* h, const moe_weights_t* w, const m
   a.gs_a0 = w->down_gs;
   a.gs_a1 = w->down_gs;
   a.act_amax = amax;
+  if (want_nvfp4_pair(s, false)) {
+    CUtensorMap sd, sh;
+    if (!make_map_sf(&sd, a.sfa0, static_cast<uint64_t>(s.E) * (s.H / 128) * (s.I / 64) * 512) ||
+        !make_map_sf(&sh, a.sfb, static_cast<uint64_t>(tiles) * (s.I / 64) * 512))
+      return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_nvfp4_pair_down(md, mh, sd, sh, a, num_sms(), stream));
+  }
   return cuda_status(moe::launch_nvfp4_down(md, mh, a, num_sms(), stream));
 }
 
@@ -625,6 +665,9 @@ bool encode_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
 }
 bool encode_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols_bytes, uint32_t box_rows) {
   return make_map_u8(map, base, rows, cols_bytes, box_rows);
+}
+bool encode_map_sf_rows(CUtensorMap* map, const void* base, uint64_t bytes, uint32_t box_rows) {
+  return make_map_sf(map, base, bytes, box_rows);
 }
 
 int check_route_args(const moe_shape_t& s, const void* x, const void* w_router, const void* topk_ids,

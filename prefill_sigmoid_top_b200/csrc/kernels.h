@@ -15,6 +15,8 @@ namespace moe {
 bool encode_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // 2-D byte tensor map [rows, cols_bytes] with boxes of box_rows x 128 bytes and the 128-byte swizzle.
 bool encode_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols_bytes, uint32_t box_rows);
+// Bytes as a [bytes / 256, 256] tensor read in unswizzled boxes of box_rows x 256 bytes (NVFP4 scale atoms).
+bool encode_map_sf_rows(CUtensorMap* map, const void* base, uint64_t bytes, uint32_t box_rows);
 
 // router_screen.cu: routing of many tokens from exact canonical logits of the candidate experts only
 // (the same ids and weights as launch_router_logits + launch_router_topk).
@@ -202,5 +204,14 @@ cudaError_t launch_nvfp4_up(const CUtensorMap& gate_codes, const CUtensorMap& up
                             const Nvfp4GemmArgs& args, int num_sms, cudaStream_t stream);
 cudaError_t launch_nvfp4_down(const CUtensorMap& down_codes, const CUtensorMap& h_codes, const Nvfp4GemmArgs& args,
                               int num_sms, cudaStream_t stream);
+
+// nvfp4_pair.cu: the same projections on 2-SM pairs; the *_sf maps read the scale atoms of the matching
+// operand as 256-byte rows (up: I % 256 == 0; down: H % 512 == 0).
+cudaError_t launch_nvfp4_pair_up(const CUtensorMap& gate_codes, const CUtensorMap& up_codes,
+                                 const CUtensorMap& x_codes, const CUtensorMap& gate_sf, const CUtensorMap& up_sf,
+                                 const CUtensorMap& x_sf, const Nvfp4GemmArgs& args, int num_sms, cudaStream_t stream);
+cudaError_t launch_nvfp4_pair_down(const CUtensorMap& down_codes, const CUtensorMap& h_codes,
+                                   const CUtensorMap& down_sf, const CUtensorMap& h_sf, const Nvfp4GemmArgs& args,
+                                   int num_sms, cudaStream_t stream);
 
 }  // namespace moe

@@ -147,6 +147,19 @@ def test_measure_calls_reject_bad_arguments():
     assert tma(FAKE, panel, 2, 4, 10, warps=0) == 1  # warps outside 1..4
     assert tma(FAKE, panel, 1, 8, 10, warps=5) == 1
     assert tma(FAKE, panel, 2, 5, 10, warps=2) == 1  # stages not a multiple of warps
+
+    def mix(buf, nbytes, m, stages, steps):
+        return L.moe_measure_tma_mix(buf, nbytes, m, stages, steps, None, ctypes.byref(moved), None)
+
+    big = 256 << 20
+    assert mix(None, big, 2, 4, 100) == 1
+    assert mix(FAKE_MIS, big, 2, 4, 100) == 1
+    assert mix(FAKE, big - 16, 2, 4, 100) == 1     # under 256 MB
+    assert mix(FAKE, big, -1, 4, 100) == 1         # mix outside 0..4
+    assert mix(FAKE, big, 5, 4, 100) == 1
+    assert mix(FAKE, big, 2, 1, 100) == 1          # stages outside 2..4
+    assert mix(FAKE, big, 2, 5, 100) == 1
+    assert mix(FAKE, big, 2, 4, 7) == 1            # fewer than 8 steps
     assert moved.value == 0
     assert L.moe_measure_hbm_read(None, 1024, None, None) == 1
     assert L.moe_measure_hbm_read(FAKE, 1000, None, None) == 1

@@ -27,3 +27,15 @@ def test_hbm_read_runs():
     moe.measure_hbm_read(buf, sink)
     torch.cuda.synchronize()
     assert int(sink.item()) == 0  # ones xor-fold to zero words: the sink is never written
+
+
+@pytest.mark.parametrize("mix,stages", [(0, 4), (1, 2), (2, 4), (3, 3), (4, 4), (4, 2)])
+def test_tma_mix_moves_what_it_reports(mix, stages):
+    buf = torch.ones(256 << 20, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    steps = 101  # several 28-step panels per CTA; not a multiple of the stage count or of the 4-step scale groups
+    moved = moe.measure_tma_mix(buf, mix, stages, steps, err)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    per_step = {0: 32768, 1: 40960, 2: 47104, 3: 47104, 4: 40960 + 3 * 8192 / 4}[mix]
+    assert moved == int(per_step * sms * steps)
+    assert moe.get_device_error(err) == 0

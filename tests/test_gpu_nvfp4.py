@@ -40,7 +40,33 @@ def _special_matrices():
     mats.append(m)
     mats.append((rng.standard_normal((64, 256)) * 50).astype(np.float32))
     mats.append(np.zeros((64, 256), np.float32))  # amax 0 -> gs 1
+    mats.append(_tie_matrix())
     return torch.tensor(np.stack(mats)).to(torch.bfloat16)
+
+
+def _bf16_step(v, up):
+    """The bf16 value next to v (a bf16-exact float32) towards +inf (up) or -inf."""
+    b = np.array([v], np.float32).view(np.uint32)[0] >> 16
+    b = b + 1 if (v >= 0) == up else b - 1
+    return np.array([b << 16], np.uint32).view(np.float32)[0]
+
+
+def _tie_matrix():
+    """Quotients exactly on the e2m1 rounding midpoints.  The matrix amax is 2688 = 6 * 448, so the global
+    scale is exactly 1; a block whose amax is 6 d, d a value of e4m3 (3 mantissa bits), gets the scale d
+    exactly, and its elements m * d (bf16-exact) divide to m for every midpoint m of the e2m1 grid: the
+    code must take the tie to even.  The blocks also hold the bf16 neighbours of those elements."""
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    m = np.zeros((64, 256), np.float32)
+    for r in range(64):
+        for b in range(16):
+            k, j = (r * 16 + b) % 13 - 6, (r + b) % 8  # d = 2^k (1 + j/8), from 2^-6 up to 120
+            d = np.float32(2.0 ** k * (1 + j / 8))
+            blk = [6 * d] + [mi * d for mi in mids] + [_bf16_step(np.float32(mi * d), i % 2 == 0)
+                                                       for i, mi in enumerate(mids)] + [-2.5 * d]
+            m[r, 16 * b:16 * b + 16] = blk
+    m[0, 0] = 2688.0  # the matrix amax (its block: d = 448)
+    return m
 
 
 def test_quantize_bitexact_against_oracle():
@@ -95,11 +121,18 @@ def _close(got, ref, rel, abs_rms):
 
 
 NVFP4_CASES = [dict(M=40, H=512, I=256, E=16, K=4, B=16), dict(M=300, H=256, I=512, E=8, K=4, B=16),
-               dict(M=7, H=768, I=256, E=32, K=6, B=32)]
+               dict(M=7, H=768, I=256, E=32, K=6, B=32),
+               dict(M=300, H=1024, I=512, E=8, K=4, B=16),   # ~150 rows per expert: two token tiles
+               dict(M=5, H=512, I=256, E=2, K=1, B=16)]      # a few rows per expert: N = 16
 
 
-@pytest.mark.parametrize("case", NVFP4_CASES, ids=lambda c: f"M{c['M']}_E{c['E']}")
-def test_nvfp4_grouped_and_layer(case):
+# "pair": the default (2-SM pair kernels wherever the weight blocks divide the expert: up I % 256 == 0,
+# down H % 512 == 0); "single": MOE_NVFP4_PAIR=0, the single-SM kernels.
+@pytest.mark.parametrize("kernels", ["pair", "single"])
+@pytest.mark.parametrize("case", NVFP4_CASES, ids=lambda c: f"M{c['M']}_H{c['H']}_E{c['E']}")
+def test_nvfp4_grouped_and_layer(case, kernels, monkeypatch):
+    if kernels == "single":
+        monkeypatch.setenv("MOE_NVFP4_PAIR", "0")
     cfg = inputs.WORKLOADS[0].with_(bias="normal", seed=case["M"] + 5, **case)
     d = inputs.make_inputs(cfg, DEV)
     shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
@@ -139,6 +172,36 @@ def test_nvfp4_grouped_and_layer(case):
     assert np.array_equal(ids.cpu().numpy(), r["ids_all"])
     ref = r["out_f64"]
     assert np.abs(bits_to_f64(bf16_bits(out)) - ref).max() <= 6e-2 * rms(ref)
+
+
+@pytest.mark.parametrize("case", NVFP4_CASES[3:4] + NVFP4_CASES[0:1] + NVFP4_CASES[4:5],
+                         ids=lambda c: f"M{c['M']}_H{c['H']}_E{c['E']}")
+def test_nvfp4_pair_equals_single_sm(case, monkeypatch):
+    """The pair kernels compute every output element from the same operands, scales and K order as the
+    single-SM kernels (one block-scaled MMA of K = 64 after another), so h and y agree bit for bit."""
+    cfg = inputs.WORKLOADS[0].with_(bias="normal", seed=case["M"] + 11, **case)
+    d = inputs.make_inputs(cfg, DEV)
+    shape = moe.Shape(cfg.M, cfg.H, cfg.I, cfg.E, cfg.K, cfg.B)
+    nw = moe.nvfp4_weights(d["w_gate"], d["w_up"], d["w_down"], shape)
+    ids, _ = moe.route(d["x"], d["w_router"], d["bias"], cfg.K)
+    plan = moe.align_block_size(ids, cfg.E, cfg.B)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+
+    def run():
+        h = moe.grouped_up_swiglu_nvfp4(d["x"], nw, plan, shape, err_flag=err)
+        y = moe.grouped_down_nvfp4(h, nw, plan, shape, err_flag=err)
+        torch.cuda.synchronize()
+        return h, y
+
+    h_p, y_p = run()
+    monkeypatch.setenv("MOE_NVFP4_PAIR", "0")
+    h_s, y_s = run()
+    assert moe.get_device_error(err) == 0
+    sorted_ids = plan["sorted_ids"].cpu().numpy()[: int(plan["num_tokens_post_padded"].item())]
+    rows = np.nonzero(sorted_ids < cfg.M * cfg.K)[0]
+    rows_t = torch.from_numpy(rows).to(DEV)
+    assert torch.equal(h_p.view(torch.int16)[rows_t], h_s.view(torch.int16)[rows_t])
+    assert torch.equal(y_p.view(torch.int16), y_s.view(torch.int16))
 
 
 def test_nvfp4_rejects_unsupported_intermediate():
