@@ -59,10 +59,12 @@ KERNEL_SOURCES = {
     "up": ["prefill_sigmoid_top_b200/csrc/gemm_bf16.cu", "prefill_sigmoid_top_b200/csrc/common.cuh"],
     "layer_fused": ["prefill_sigmoid_top_b200/csrc/layer_fused.cu", "prefill_sigmoid_top_b200/csrc/common.cuh",
                     "prefill_sigmoid_top_b200/csrc/router_dot.cuh"],
-    "pair_up": ["prefill_sigmoid_top_b200/csrc/gemm_pair.cu", "prefill_sigmoid_top_b200/csrc/common.cuh",
-                "prefill_sigmoid_top_b200/csrc/tile_list.cuh"],
+    "pair_up": ["prefill_sigmoid_top_b200/csrc/gemm_pair.cu", "prefill_sigmoid_top_b200/csrc/pair_ptx.cuh",
+                "prefill_sigmoid_top_b200/csrc/common.cuh", "prefill_sigmoid_top_b200/csrc/tile_list.cuh"],
     "nvfp4_up": ["prefill_sigmoid_top_b200/csrc/nvfp4.cu", "prefill_sigmoid_top_b200/csrc/common.cuh",
                  "prefill_sigmoid_top_b200/csrc/tile_list.cuh"],
+    "nvfp4_pair_up": ["prefill_sigmoid_top_b200/csrc/nvfp4_pair.cu", "prefill_sigmoid_top_b200/csrc/pair_ptx.cuh",
+                      "prefill_sigmoid_top_b200/csrc/common.cuh", "prefill_sigmoid_top_b200/csrc/tile_list.cuh"],
 }
 
 
@@ -543,10 +545,18 @@ def measure_workload(cfg, args, dev, world, rank, want_cpu, read_ceiling_box):
                "traffic": ncu_traffic("layer_fused")}
     else:
         pair = (not nvfp4) and cid in (2, 3)
-        name = ": pair_gemm_kernel<up>" if pair else (": persistent_nvfp4_kernel<up>" if nvfp4 else "")
+        # the NVFP4 up projection runs on 2-SM pairs when I is a multiple of 256, unless MOE_NVFP4_PAIR=0
+        nvfp4_pair = nvfp4 and cfg.I % 256 == 0 and os.environ.get("MOE_NVFP4_PAIR") != "0"
+        if pair:
+            name, key = ": pair_gemm_kernel<up>", "pair_up"
+        elif nvfp4:
+            name, key = ((": nvfp4_pair_kernel<up>", "nvfp4_pair_up") if nvfp4_pair
+                         else (": persistent_nvfp4_kernel<up>", "nvfp4_up"))
+        else:
+            name, key = "", None
         dom = {"kernel": "grouped_up_swiglu (staged pass)" + name,
                "achieved": up_achieved, "algorithmic_bytes": ab["up"],
-               "traffic": ncu_traffic("pair_up") if pair else (ncu_traffic("nvfp4_up") if nvfp4 else None)}
+               "traffic": ncu_traffic(key) if key else None}
     dom.update(bound="hbm", peak=hbm_peak, unit="GB/s", frac=dom["achieved"] / hbm_peak, peak_source=peak_kind)
     if read_ceiling_box.get("gbs"):
         dom["read_ceiling_gbs"] = read_ceiling_box["gbs"]
