@@ -50,9 +50,11 @@ NCU_TRAFFIC = {
     (1, "layer_fused"): (8_382_036_224, "9c39ca834ce5fa81"),
     # batch M=512 and prefill M=2048: the up projection (2-SM pair kernel) captured at full size, one pass
     # (dram__bytes_read.sum + dram__bytes_write.sum of one launch)
-    (2, "pair_up"): (15_305_074_944, "5c0cd642d8591f67"),
-    (3, "pair_up"): (16_934_910_208, "5c0cd642d8591f67"),
-    # NVFP4 M=1000: the block-scaled up projection captured at full size, one pass
+    (2, "pair_up"): (15_296_836_864, "f133d19d41b4abbf"),
+    (3, "pair_up"): (16_907_707_648, "f133d19d41b4abbf"),
+    # NVFP4 M=1000: the block-scaled up projection captured at full size, one pass: on 2-SM pairs (the
+    # default) and on single SMs (MOE_NVFP4_PAIR=0)
+    (4, "nvfp4_pair_up"): (4_565_486_080, "c09c4a0689ec51c0"),
     (4, "nvfp4_up"): (4_656_227_584, "cc73a5d8c3d56c67"),
 }
 KERNEL_SOURCES = {
