@@ -176,7 +176,10 @@ MOE_API size_t moe_align_capacity(moe_shape_t s); /* M*top_k + E*(block_size-1) 
  * contiguous rows; without it the rows are gathered inside the GEMM.  Both
  * give the same result.  MOE_W_NVFP4: x is quantised on the fly (global scale
  * from the amax over all of x) into ws (required), and the accumulators are
- * scaled by gs_gate[e] * gs_x and gs_up[e] * gs_x before SwiGLU. */
+ * scaled by gs_gate[e] * gs_x and gs_up[e] * gs_x before SwiGLU; the block-
+ * scaled GEMM runs on 2-SM pairs (cta_group::2) when I % 256 == 0 and on
+ * single SMs otherwise or with MOE_NVFP4_PAIR=0 in the environment, with the
+ * same bits either way. */
 MOE_API moe_status_t moe_grouped_up_swiglu(const moe_bf16_t* x, const moe_weights_t* w, const moe_plan_t* plan,
                                    moe_shape_t s, moe_bf16_t* h, void* ws, size_t ws_bytes, int32_t* err_flag,
                                    moe_stream_t stream);
@@ -212,7 +215,8 @@ MOE_API moe_status_t moe_grouped_up_swiglu_routed(const moe_bf16_t* x, const moe
  * h: bf16 [cap, I]; y: bf16 [M*top_k, H] (slot-major: y[t, k, :]).
  * MOE_W_NVFP4: h is quantised on the fly (global scale from the amax over the
  * real plan rows of h) into ws, moe_down_workspace_size(s, MOE_W_NVFP4) bytes
- * (required); the accumulators are scaled by gs_down[e] * gs_h. */
+ * (required); the accumulators are scaled by gs_down[e] * gs_h; 2-SM pairs
+ * when H % 512 == 0 (MOE_NVFP4_PAIR=0: single SMs), the same bits either way. */
 MOE_API moe_status_t moe_grouped_down(const moe_bf16_t* h, const moe_weights_t* w, const moe_plan_t* plan,
                               moe_shape_t s, moe_bf16_t* y, void* ws, size_t ws_bytes, int32_t* err_flag,
                               moe_stream_t stream);
